@@ -1,0 +1,309 @@
+"""Benchmark: Sol-Attn forward on one B200 per rank (effective TFLOP/s and ms per call).
+
+Workload (default ``s64k``): B=1, H=32, d=128, N=65536 tokens (16x64x64 latent grid, t-major),
+seeded BF16 Gaussian-random-field Q/K/V, tau tuned so 90 % of (query-block, key-block) pairs are
+not exact.  A step is one ``sol_attn_fwd`` call: block summaries, threshold statistics, routing and
+the fused attention kernel.  Inputs (3 x 537 MB) are larger than the 126 MB L2, so no flush is
+needed between steps.
+
+Effective FLOPs per step: 4 d (N^2 / Nb^2) E  for the exact pairs E (= 4 N^2 d H (1 - sp)) plus
+4 d 64 (P - E) for the surrogate pairs, with P = B H Nb^2 and the realised sparsity sp reported by
+the library.  ``value`` is the aggregate over all ranks (weak scaling: every rank runs its own
+batch element on its own GPU; no data-path collective).
+
+``--impl reference`` times the FP64 CPU oracle (the only reference implementation that exists for
+this method) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn fwd ms & effective TFLOP/s vs BF16 peak, 32 heads d128, 32K–128K tok"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="s64k")
+    ap.add_argument("--cpu-sample-blocks", type=int, default=24,
+                    help="query blocks of one head the CPU oracle baseline evaluates")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_PATH):
+        with open(PEAKS_PATH) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def effective_flops(B, N, H, exact_pairs, total_pairs, d=128):
+    Nb = (N + 63) // 64
+    per_exact = 4.0 * d * (N / Nb) ** 2          # = 4 * 64 * 64 * d for full blocks
+    per_surrogate = 4.0 * d * (N / Nb)           # one pooled key per unselected block and query
+    exact_flops = per_exact * exact_pairs
+    return exact_flops + per_surrogate * (total_pairs - exact_pairs), exact_flops
+
+
+# ------------------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(device_index), "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                     util=float(parts[4]), hw=parts[6], hwt=parts[7], swt=parts[8], pcap=parts[9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        loaded = [r for r in rows if r["util"] >= 50] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ------------------------------------------------------------------------------------ CPU baseline
+
+def cpu_baseline(workload, n_blocks: int, q=None, k=None, v=None):
+    """The FP64 oracle, as it stands, on one head: full summaries / thresholds for that head and
+    ``n_blocks`` seeded query blocks.  Returns the oracle's effective TFLOP/s on that sample."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import sol_attn_oracle as orc
+
+    if q is None:
+        q, k, v = workload.make_inputs("cpu")
+    tau = workload.resolved_tau()
+    Nb = orc.num_blocks(workload.N)
+    blocks = sorted(np.random.default_rng(7).choice(Nb, size=min(n_blocks, Nb), replace=False).tolist())
+    fn = getattr(orc, workload.entry)
+    t0 = time.perf_counter()
+    r = fn(q, k, v, tau, workload.sink_start, workload.sink_tokens, qblocks=blocks, heads=[(0, 0)])
+    dt = time.perf_counter() - t0
+    rows = r["mask"][0, 0][blocks]
+    exact = int(rows.sum())
+    total = rows.size
+    flops, _ = effective_flops(1, workload.N, 1, exact, total)
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{workload.name}: head 0 of {workload.H}, {len(blocks)} of {Nb} query blocks "
+                      f"(summaries and thresholds of that head in full), FP64 numpy, {dt:.1f} s",
+            "seconds": dt}
+
+
+# ---------------------------------------------------------------------------------------------- main
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from block_sparse_attention_sum_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        base = cpu_baseline(w, args.cpu_sample_blocks)
+        line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": 1, "warmup": 0, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "seq_len": w.N,
+                           "global_batch": w.B, "parallelism": "cpu"},
+                "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": base["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_attention_sum_b200 import sol_attn as sa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # inputs: seeded on the CPU (deterministic), pinned for the end-to-end leg; each rank its own batch element
+    from block_sparse_attention_sum_b200.inputs import grf_qkv, iid_qkv
+
+    seed = w.seed + 100 * rank
+    if w.kind == "grf":
+        qh, kh, vh = grf_qkv(w.B, w.H, w.grid, seed_base=seed)
+    else:
+        qh, kh, vh = iid_qkv(w.B, w.N, w.H, seed=seed)
+    qh, kh, vh = (t.pin_memory() for t in (qh, kh, vh))
+    q, k, v = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
+    out = torch.empty_like(q)
+    tau = w.resolved_tau()
+    fn = sa.sol_attn_fwd if w.entry == "sol_attn" else sa.sol_attn2_fwd
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fn(q, k, v, tau, w.sink_start, w.sink_tokens, out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0, "device status after warm-up"
+    exact, total, _, _ = sa.last_stats()
+    launches_per_step = sa.last_launch_count()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- timed region: inputs resident in HBM
+    clocks = ClockSampler(local_rank)
+    sa.set_kernel_timing(True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+    elapsed_ms = e0.elapsed_time(e1)
+    kernel_ms = sa.kernel_ms_sum(min(args.steps, 256)) / min(args.steps, 256)
+    sa.set_kernel_timing(False)
+    assert sa.get_device_status() == 0, "device status after the timed region"
+
+    t = torch.tensor([elapsed_ms, kernel_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, kernel_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed_ms / args.steps
+    flops_step, exact_flops_step = effective_flops(w.B, w.N, w.H, exact, total)
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+    sp = 1.0 - exact / total
+
+    # ---- end to end through the public API with host buffers (H2D inputs, D2H output each step)
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty_like(qh).pin_memory()
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t2 = torch.tensor([a.elapsed_time(b) / e2e_steps], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t2[0])
+        e2e = {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 3 * qh.numel() * qh.element_size(),
+               "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": e2e_steps}
+
+    peaks = load_peaks()
+    peak_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    peak_burst = float(peaks["bf16_tflops"])
+    achieved = flops_step / (kernel_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sust, "unit": "TFLOP/s",
+                "frac": achieved / peak_sust, "traffic": None,
+                "kernel": "attn_fwd_kernel<false> (fused routing + attention)",
+                "kernel_ms": kernel_ms, "peak_kind": f"bf16 dense sustained ({peaks['source']})",
+                "frac_of_burst": achieved / peak_burst}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d=128 GRF t-major {w.grid.T}x{w.grid.Y}x{w.grid.X}"
+                                   if w.grid else w.name,
+                       "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "tau": tau,
+                       "target_sparsity": w.target_sparsity, "realised_sparsity": sp,
+                       "parallelism": f"independent replicas x{world} (head/batch sharding, no exchange)",
+                       "l2": "inputs 1.6 GB per rank > 126 MB L2; no flush"},
+            "frac_of_peak": value / world / peak_burst, "frac_of_sustained_peak": value / world / peak_sust,
+            "exact_only_tflops": exact_flops_step * world / (ms_per_step * 1e-3) / 1e12,
+            "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clock_info}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(w, args.cpu_sample_blocks, qh, kh, vh)
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,451 @@
+// Host side of the C ABI declared in include/sol_attn.h: argument validation, the per-device
+// workspace, TMA descriptors and the launch sequence.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "attn_fwd.cuh"
+#include "common.cuh"
+#include "ptx.cuh"
+#include "sol_attn.h"
+
+namespace sol {
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool checked = false;
+  bool usable = false;
+  void* ws = nullptr;      // workspace
+  size_t ws_bytes = 0;
+  int* status = nullptr;   // device status word
+  unsigned long long* stats = nullptr;
+  cudaEvent_t done = nullptr;   // completion of the previous call (cross-stream ordering)
+  static constexpr int kRing = 256;
+  cudaEvent_t t0[kRing] = {}, t1[kRing] = {};
+  int timed_calls = 0;      // timed launches since timing was enabled
+  cudaStream_t last_stream = nullptr;
+  long long last_total_pairs = 0;
+  int last_launches = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+bool g_timing = false;
+int g_last_device = -1;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode() {
+  if (g_encode) return SOL_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return fail(SOL_ERR_DEVICE, "cuTensorMapEncodeTiled is unavailable");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return SOL_OK;
+}
+
+int device_state(DeviceState** out, int* dev_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(SOL_ERR_DEVICE, "no current CUDA device");
+  DeviceState& d = g_dev[dev];
+  if (!d.checked) {
+    d.checked = true;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return fail(SOL_ERR_DEVICE, "cudaGetDeviceProperties failed");
+    d.usable = prop.major == 10 && prop.minor == 0;
+    if (d.usable) {
+      if (cudaMalloc(&d.status, sizeof(int)) != cudaSuccess ||
+          cudaMalloc(&d.stats, 4 * sizeof(unsigned long long)) != cudaSuccess ||
+          cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess ||
+          cudaEventCreateWithFlags(&d.done, cudaEventDisableTiming) != cudaSuccess) {
+        d.checked = false;
+        return fail(SOL_ERR_ALLOC, "device state allocation failed");
+      }
+    }
+  }
+  if (!d.usable) return fail(SOL_ERR_DEVICE, "device %d is not an sm_100 (B200-class) GPU", dev);
+  *out = &d;
+  *dev_out = dev;
+  return SOL_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Carves the workspace into the buffers of one call; returns the bytes needed when base == nullptr.
+size_t carve(const Shape& s, bool sol2, char* base, Work* w) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes, 256);
+    return p;
+  };
+  const size_t bh = (size_t)s.BH, nb = (size_t)s.Nb, d = kHeadDim;
+  Work t{};
+  t.qbar = reinterpret_cast<float*>(take(bh * nb * d * 4));
+  t.kbar = reinterpret_cast<float*>(take(bh * nb * d * 4));
+  t.kbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.vbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.kcov = reinterpret_cast<float*>(take(bh * d * d * 4));
+  t.kmean = reinterpret_cast<double*>(take(bh * d * 8));
+  t.thresh = reinterpret_cast<float*>(take(bh * nb * 4));
+  t.mask = reinterpret_cast<uint32_t*>(take(bh * nb * s.Nw * 4));
+  t.rowcount = reinterpret_cast<int*>(take(bh * nb * 4));
+  if (sol2) {
+    const size_t na = (size_t)s.Na;
+    t.qanchor = reinterpret_cast<float*>(take(bh * na * d * 4));
+    t.qdir = reinterpret_cast<float*>(take(bh * d * 4));
+    t.gk = reinterpret_cast<float*>(take(bh * nb * 2 * d * 4));
+    t.gv = reinterpret_cast<float*>(take(bh * nb * 2 * d * 4));
+    t.gcount = reinterpret_cast<int*>(take(bh * nb * 2 * 4));
+    t.tail_logz = reinterpret_cast<float*>(take(bh * na * 4));
+    t.tail_mu = reinterpret_cast<float*>(take(bh * na * d * 4));
+    t.tail_nu = reinterpret_cast<float*>(take(bh * na * d * 4));
+  }
+  if (w) *w = t;
+  return off;
+}
+
+int ensure_workspace(DeviceState& d, size_t bytes) {
+  if (d.ws_bytes >= bytes) return SOL_OK;
+  if (d.ws) {
+    cudaDeviceSynchronize();
+    cudaFree(d.ws);
+    d.ws = nullptr;
+    d.ws_bytes = 0;
+  }
+  const size_t grow = align_up(bytes + bytes / 8, 1 << 20);
+  if (cudaMalloc(&d.ws, grow) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SOL_ERR_ALLOC, "workspace allocation of %zu bytes failed", grow);
+  }
+  d.ws_bytes = grow;
+  return SOL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int validate(const void* q, const void* k, const void* v, const void* out, bool need_v_out, int B, int N, int H,
+             float tau, int sink_start, int sink_tokens) {
+  if (!q || !k || (need_v_out && (!v || !out))) return fail(SOL_ERR_NULL, "q, k, v and out must be non-NULL");
+  if (B <= 0 || N <= 0 || H <= 0) return fail(SOL_ERR_SHAPE, "B, N, H must be positive (got %d, %d, %d)", B, N, H);
+  const long long elems = (long long)B * N * H * kHeadDim;
+  if (elems > (1ll << 40) || (long long)B * H > (1ll << 24) || N > (1 << 30))
+    return fail(SOL_ERR_SHAPE, "sizes out of the supported range");
+  if (!std::isfinite(tau)) return fail(SOL_ERR_TAU, "tau must be finite");
+  if (sink_tokens > 0 && sink_start >= N) return fail(SOL_ERR_SINK, "sink_start (%d) must be < N (%d)", sink_start, N);
+  if (!aligned16(q) || !aligned16(k) || (need_v_out && (!aligned16(v) || !aligned16(out))))
+    return fail(SOL_ERR_ALIGN, "tensor pointers must be 16-byte aligned");
+  if (need_v_out) {
+    const size_t bytes = (size_t)elems * 2;
+    if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) || overlaps(out, bytes, v, bytes))
+      return fail(SOL_ERR_ALIGN, "out must not overlap q, k or v");
+  }
+  return SOL_OK;
+}
+
+// Key blocks overlapping the sink range, as an inclusive block interval (b0 > b1: no sink).
+void sink_blocks(int N, int sink_start, int sink_tokens, int* b0, int* b1) {
+  *b0 = 1;
+  *b1 = 0;
+  if (sink_tokens <= 0) return;
+  long long start = sink_start >= 0 ? sink_start : (long long)N - sink_tokens;
+  long long end = start + sink_tokens;
+  if (start < 0) start = 0;
+  if (end > N) end = N;
+  if (end <= start) return;
+  *b0 = (int)(start / kBlock);
+  *b1 = (int)((end - 1) / kBlock);
+}
+
+int encode_bthd(CUtensorMap* m, const void* base, const Shape& s) {
+  const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)s.H, (cuuint64_t)s.N, (cuuint64_t)s.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)s.H * kHeadDim * 2,
+                                 (cuuint64_t)s.N * s.H * kHeadDim * 2};
+  const cuuint32_t box[4] = {64, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOL_OK : fail(SOL_ERR_LAUNCH, "cuTensorMapEncodeTiled (BTHD) failed: %d", (int)r);
+}
+
+int encode_pooled(CUtensorMap* m, const void* base, const Shape& s) {
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)s.Nb, (cuuint64_t)s.BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)s.Nb * kHeadDim * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOL_OK : fail(SOL_ERR_LAUNCH, "cuTensorMapEncodeTiled (pooled) failed: %d", (int)r);
+}
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "%s: %s", what, cudaGetErrorString(e));
+  return SOL_OK;
+}
+
+// Routing prefix shared by all entry points: summaries, threshold statistics, thresholds, bitmask.
+int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                const Shape& s, const Work& w, float tau, int sink_start, int sink_tokens, bool anchors,
+                cudaStream_t st, int* launches) {
+  int sb0, sb1;
+  sink_blocks(s.N, sink_start, sink_tokens, &sb0, &sb1);
+  const unsigned long long init[3] = {0ull, ~0ull, 0ull};
+  (void)init;
+  if (cudaMemsetAsync(d.stats, 0, sizeof(unsigned long long), st) != cudaSuccess ||
+      cudaMemsetAsync(d.stats + 1, 0xff, sizeof(unsigned long long), st) != cudaSuccess ||
+      cudaMemsetAsync(d.stats + 2, 0, sizeof(unsigned long long), st) != cudaSuccess)
+    return fail(SOL_ERR_LAUNCH, "stats reset failed");
+  Work ww = w;
+  ww.stats = d.stats;
+  launch_summary(q, k, v, s, ww, anchors, st);
+  launch_kstats(s, ww, st);
+  launch_thresh(s, ww, tau, st);
+  launch_route(s, ww, sb0, sb1, st);
+  *launches += 4;
+  d.last_total_pairs = (long long)s.BH * s.Nb * s.Nb;
+  return check_launch("routing kernels");
+}
+
+int forward(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau, int sink_start,
+            int sink_tokens, void* stream, bool sol2) {
+  int rc = validate(q, k, v, out, true, B, N, H, tau, sink_start, sink_tokens);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* d;
+  int dev;
+  if ((rc = device_state(&d, &dev))) return rc;
+  if ((rc = get_encode())) return rc;
+  const Shape s = make_shape(B, N, H);
+  Work w;
+  const size_t need = carve(s, sol2, nullptr, nullptr);
+  if ((rc = ensure_workspace(*d, need))) return rc;
+  carve(s, sol2, static_cast<char*>(d->ws), &w);
+  w.stats = d->stats;
+
+  CUtensorMap maps[5];
+  if ((rc = encode_bthd(&maps[0], q, s)) || (rc = encode_bthd(&maps[1], k, s)) || (rc = encode_bthd(&maps[2], v, s)) ||
+      (rc = encode_pooled(&maps[3], w.kbar_h, s)) || (rc = encode_pooled(&maps[4], w.vbar_h, s)))
+    return rc;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamWaitEvent(st, d->done, 0) != cudaSuccess) return fail(SOL_ERR_LAUNCH, "cudaStreamWaitEvent failed");
+  int launches = 0;
+  const auto* qh = static_cast<const __nv_bfloat16*>(q);
+  const auto* kh = static_cast<const __nv_bfloat16*>(k);
+  const auto* vh = static_cast<const __nv_bfloat16*>(v);
+  if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, st, &launches))) return rc;
+  if (sol2) {
+    launch_groups(qh, kh, vh, s, w, st);
+    launch_anchor_tail(s, w, st);
+    launches += 3;
+    if ((rc = check_launch("Sol-Attn2 tail kernels"))) return rc;
+  }
+  FwdParams p{};
+  p.N = N;
+  p.H = H;
+  p.Nb = s.Nb;
+  p.Nw = s.Nw;
+  p.Na = s.Na;
+  p.QT = s.QT;
+  p.mask = w.mask;
+  p.order = nullptr;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = d->status;
+  p.qanchor = w.qanchor;
+  p.tail_logz = w.tail_logz;
+  p.tail_mu = w.tail_mu;
+  p.tail_nu = w.tail_nu;
+  const int slot = d->timed_calls % DeviceState::kRing;
+  if (g_timing) {
+    if (!d->t0[slot] && (cudaEventCreate(&d->t0[slot]) != cudaSuccess || cudaEventCreate(&d->t1[slot]) != cudaSuccess))
+      return fail(SOL_ERR_LAUNCH, "timing event creation failed");
+    cudaEventRecord(d->t0[slot], st);
+  }
+  cudaError_t e = launch_attn_fwd(maps, p, s.BH * s.QT, sol2, st);
+  if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "fused attention launch: %s", cudaGetErrorString(e));
+  if (g_timing) {
+    cudaEventRecord(d->t1[slot], st);
+    ++d->timed_calls;
+  }
+  launches += 1;
+  cudaEventRecord(d->done, st);
+  d->last_stream = st;
+  d->last_launches = launches;
+  g_last_device = dev;
+  return SOL_OK;
+}
+
+}  // namespace
+}  // namespace sol
+
+using namespace sol;
+
+extern "C" {
+
+int sol_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                 int sink_start, int sink_tokens, void* stream) {
+  g_err[0] = 0;
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, stream, false);
+}
+
+int sol_attn2_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                  int sink_start, int sink_tokens, void* stream) {
+  g_err[0] = 0;
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, stream, true);
+}
+
+const char* sol_attn_last_error(void) { return g_err; }
+
+int sol_attn_get_device_status(void* stream) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* d;
+  int dev;
+  int rc = device_state(&d, &dev);
+  if (rc) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(SOL_ERR_LAUNCH, "stream synchronisation failed: %s", cudaGetErrorString(cudaGetLastError()));
+  int h = 0;
+  if (cudaMemcpy(&h, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(d->status, 0, sizeof(int)) != cudaSuccess)
+    return fail(SOL_ERR_LAUNCH, "status read failed");
+  if (h == kDevTimeout) return fail(SOL_ERR_TIMEOUT, "a bounded wait inside a kernel ran out");
+  return SOL_OK;
+}
+
+int sol_attn_debug_route(const void* q, const void* k, int B, int N, int H, float tau, int sink_start,
+                         int sink_tokens, unsigned char* mask, float* thresh, void* stream) {
+  g_err[0] = 0;
+  int rc = validate(q, k, nullptr, nullptr, false, B, N, H, tau, sink_start, sink_tokens);
+  if (rc) return rc;
+  if (!mask) return fail(SOL_ERR_NULL, "mask must be non-NULL");
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* d;
+  int dev;
+  if ((rc = device_state(&d, &dev))) return rc;
+  const Shape s = make_shape(B, N, H);
+  Work w;
+  if ((rc = ensure_workspace(*d, carve(s, false, nullptr, nullptr)))) return rc;
+  carve(s, false, static_cast<char*>(d->ws), &w);
+  w.stats = d->stats;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStreamWaitEvent(st, d->done, 0);
+  int launches = 0;
+  // the summary kernel reads v as well; pass k, whose summaries are simply discarded
+  if ((rc = run_routing(*d, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                        static_cast<const __nv_bfloat16*>(k), s, w, tau, sink_start, sink_tokens, false, st,
+                        &launches)))
+    return rc;
+  launch_expand_mask(s, w, mask, st);
+  if (thresh) cudaMemcpyAsync(thresh, w.thresh, (size_t)s.BH * s.Nb * sizeof(float), cudaMemcpyDeviceToDevice, st);
+  if ((rc = check_launch("route introspection"))) return rc;
+  cudaEventRecord(d->done, st);
+  d->last_stream = st;
+  d->last_launches = launches + 1;
+  g_last_device = dev;
+  return SOL_OK;
+}
+
+int sol_attn_last_stats(long long* exact_pairs, long long* total_pairs, int* min_row, int* max_row) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_last_device < 0) return fail(SOL_ERR_LAUNCH, "no call has run yet");
+  DeviceState& d = g_dev[g_last_device];
+  int cur = -1;
+  cudaGetDevice(&cur);
+  cudaSetDevice(g_last_device);
+  unsigned long long h[3] = {0, 0, 0};
+  cudaError_t e = cudaStreamSynchronize(d.last_stream);
+  if (e == cudaSuccess) e = cudaMemcpy(h, d.stats, sizeof(h), cudaMemcpyDeviceToHost);
+  cudaSetDevice(cur);
+  if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "stats read failed: %s", cudaGetErrorString(e));
+  if (exact_pairs) *exact_pairs = (long long)h[0];
+  if (total_pairs) *total_pairs = d.last_total_pairs;
+  if (min_row) *min_row = (int)h[1];
+  if (max_row) *max_row = (int)h[2];
+  return SOL_OK;
+}
+
+int sol_attn_set_kernel_timing(int enable) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_timing = enable != 0;
+  if (g_timing)
+    for (auto& d : g_dev) d.timed_calls = 0;
+  return SOL_OK;
+}
+
+static float kernel_ms_sum_locked(int n) {
+  if (g_last_device < 0) return -1.f;
+  DeviceState& d = g_dev[g_last_device];
+  if (n <= 0 || n > d.timed_calls || n > DeviceState::kRing) return -1.f;
+  double total = 0.0;
+  for (int i = d.timed_calls - n; i < d.timed_calls; ++i) {
+    const int slot = i % DeviceState::kRing;
+    float ms = -1.f;
+    if (cudaEventSynchronize(d.t1[slot]) != cudaSuccess || cudaEventElapsedTime(&ms, d.t0[slot], d.t1[slot]) != cudaSuccess)
+      return -1.f;
+    total += ms;
+  }
+  return (float)total;
+}
+
+float sol_attn_last_kernel_ms(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return kernel_ms_sum_locked(1);
+}
+
+float sol_attn_kernel_ms_sum(int n) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return kernel_ms_sum_locked(n);
+}
+
+int sol_attn_last_launch_count(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return g_last_device < 0 ? 0 : g_dev[g_last_device].last_launches;
+}
+
+void sol_attn_release_workspace(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = -1;
+  cudaGetDevice(&cur);
+  for (int i = 0; i < kMaxDevices; ++i) {
+    DeviceState& d = g_dev[i];
+    if (!d.ws) continue;
+    cudaSetDevice(i);
+    cudaDeviceSynchronize();
+    cudaFree(d.ws);
+    d.ws = nullptr;
+    d.ws_bytes = 0;
+  }
+  if (cur >= 0) cudaSetDevice(cur);
+}
+
+}  // extern "C"

@@ -1,0 +1,490 @@
+// Fused Sol-Attn forward for sm_100a: exact 64x64 blocks and pooled surrogate tiles through one
+// tcgen05 pipeline with one online-softmax state per query row.
+//
+// Sol-Attn paper (arXiv 2607.24027), section 3.2: "Chunk-wise On-the-Fly Thresholding",
+// "Proxy-Score Reuse as Approximate Correction" (token-to-block scores reused for the unselected
+// blocks, selected columns masked), "Hardware-Aligned Implementation" (Q_i staged in shared memory,
+// one online-softmax state, K/V loaded only for routed blocks; pooled key KC and summed value VC).
+// Sol-Attn2 draft, "Routing and complementary approximation" (tail merged in the epilogue).
+//
+// B200 design (differs from the paper's nested loop, see the design notes):
+//  * A work unit is a 128-row query tile = two adjacent 64-token query blocks, so every tcgen05.mma
+//    runs at M = 128.  The unit walks the union of the two blocks' exact sets, two key blocks
+//    (128 keys) per tile; columns of a block that is exact for only one half are masked for the
+//    other half, whose surrogate then covers that block.
+//  * Surrogate tiles: 128 pooled keys Kbar_j (BF16) as the B operand of S = Q K^T and the value
+//    means Vbar_j as the B operand of O += P V, with a per-column log-mass bias log2(n_j) and -inf
+//    for the columns that are exact for the row's block.  n_j exp(a_j) and exp(a_j) n_j Vbar_j =
+//    exp(a_j) Vhat_j are exactly the surrogate's denominator and numerator terms.
+//  * Warp roles: warp 0 TMA producer (derives the tile list from the routing bitmask), warp 1 TMEM
+//    owner and MMA issuer, warps 4-7 softmax / O-correction / epilogue (one thread per query row,
+//    TMEM lane = row).  S is double-buffered in TMEM; O accumulates in TMEM.
+//  * Online softmax in base 2 with a lazily updated reference max: O and l are rescaled only when a
+//    row's max grows by more than 2^8, which keeps every probability <= 256.
+#include <cuda.h>
+#include <cfloat>
+
+#include "attn_fwd.cuh"
+#include "ptx.cuh"
+
+namespace sol {
+
+namespace {
+
+constexpr int kStages = 2;
+constexpr uint32_t kTileBytes = 128 * 64 * 2;  // one 128-row x 64-column BF16 box pair half (16 KB)
+constexpr uint32_t kBoxBytes = 64 * 64 * 2;    // one 64-row x 64-column BF16 TMA box (8 KB)
+
+enum : uint32_t { kTilePair = 0, kTileSingle = 1, kTilePooled = 2 };
+
+struct TileDesc {
+  uint32_t kind;
+  int j0, j1;       // key blocks (exact tiles) or the pooled chunk index (j0)
+  uint32_t flags;   // bit 0/1: j0 exact for half 0/1; bit 2/3: j1 exact for half 0/1; bit 8: last tile
+};
+
+struct __align__(1024) FwdSmem {
+  __nv_bfloat16 q[2][128 * 64];            // [d half][128 rows x 64], K-major SW128
+  __nv_bfloat16 k[kStages][2][128 * 64];   // [stage][d half][128 keys x 64]
+  __nv_bfloat16 v[kStages][2][128 * 64];
+  __nv_bfloat16 p[2][128 * 64];            // [key half][128 rows x 64 keys]
+  TileDesc desc[kStages];
+  uint64_t full[kStages], empty[kStages];
+  uint64_t qfull, sfull[2], sfree[2], pready, pvdone, mmadone;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = sizeof(FwdSmem) + 1024;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void set_timeout(int* status) { atomicExch(status, kDevTimeout); }
+
+}  // namespace
+
+template <bool kSol2>
+__global__ void __launch_bounds__(256, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+                    const __grid_constant__ CUtensorMap tm_vp, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem& sm = *reinterpret_cast<FwdSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort = &sm.abort;
+
+  const int unit = p.order ? p.order[blockIdx.x] : (int)blockIdx.x;
+  const int bh = unit / p.QT, qt = unit % p.QT;
+  const int b = bh / p.H, h = bh % p.H;
+  const int qb0 = 2 * qt;
+  const bool has_hi = qb0 + 1 < p.Nb;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.qfull, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.sfull[i], 1);
+      mbar_init(&sm.sfree[i], 128);
+    }
+    mbar_init(&sm.pready, 128);
+    mbar_init(&sm.pvdone, 1);
+    mbar_init(&sm.mmadone, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ----------------------------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      if (!kSol2) {
+        tma_prefetch_desc(&tm_kp);
+        tma_prefetch_desc(&tm_vp);
+      }
+      mbar_arrive_expect_tx(&sm.qfull, 4 * kBoxBytes);
+      for (int hf = 0; hf < 2; ++hf)
+        for (int dh = 0; dh < 2; ++dh)
+          tma_load_4d(&sm.q[dh][hf * 64 * 64], &tm_q, &sm.qfull, 64 * dh, h, 64 * (qb0 + hf), b);
+
+      const uint32_t* row0 = p.mask + ((size_t)bh * p.Nb + qb0) * p.Nw;
+      const uint32_t* row1 = row0 + p.Nw;
+      int t = 0;
+      bool ok = true;
+      TileDesc prev;
+      bool have_prev = false;
+      auto issue = [&](TileDesc d) {
+        const int s = t % kStages;
+        if (t >= kStages && !mbar_wait(&sm.empty[s], ((t / kStages) - 1) & 1, abort)) {
+          ok = false;
+          return;
+        }
+        sm.desc[s] = d;
+        if (d.kind == kTilePooled) {
+          mbar_arrive_expect_tx(&sm.full[s], 4 * kTileBytes);
+          for (int dh = 0; dh < 2; ++dh) {
+            tma_load_3d(&sm.k[s][dh][0], &tm_kp, &sm.full[s], 64 * dh, 128 * d.j0, bh);
+            tma_load_3d(&sm.v[s][dh][0], &tm_vp, &sm.full[s], 64 * dh, 128 * d.j0, bh);
+          }
+        } else {
+          const int nblk = d.kind == kTilePair ? 2 : 1;
+          mbar_arrive_expect_tx(&sm.full[s], 4 * kBoxBytes * nblk);
+          for (int slot = 0; slot < nblk; ++slot) {
+            const int j = slot ? d.j1 : d.j0;
+            for (int dh = 0; dh < 2; ++dh) {
+              tma_load_4d(&sm.k[s][dh][slot * 64 * 64], &tm_k, &sm.full[s], 64 * dh, h, 64 * j, b);
+              tma_load_4d(&sm.v[s][dh][slot * 64 * 64], &tm_v, &sm.full[s], 64 * dh, h, 64 * j, b);
+            }
+          }
+        }
+        ++t;
+      };
+      auto push = [&](TileDesc d) {
+        if (have_prev && ok) issue(prev);
+        prev = d;
+        have_prev = true;
+      };
+      // exact tiles: the union of the two rows' exact blocks, in increasing order, two per tile
+      int pend = -1;
+      uint32_t pend_fl = 0;
+      for (int wd = 0; wd < p.Nw && ok; ++wd) {
+        const uint32_t a = row0[wd];
+        const uint32_t c = has_hi ? row1[wd] : 0u;
+        uint32_t u = a | c;
+        while (u && ok) {
+          const int bit = __ffs(u) - 1;
+          u &= u - 1;
+          const int j = 32 * wd + bit;
+          const uint32_t fl = ((a >> bit) & 1u) | (((c >> bit) & 1u) << 1);
+          if (pend < 0) {
+            pend = j;
+            pend_fl = fl;
+          } else {
+            push(TileDesc{kTilePair, pend, j, pend_fl | (fl << 2)});
+            pend = -1;
+          }
+        }
+      }
+      if (pend >= 0 && ok) push(TileDesc{kTileSingle, pend, pend, pend_fl});
+      if (!kSol2) {
+        // surrogate tiles: 128 pooled keys each; skip chunks that are exact for both rows
+        const int nchunk = (p.Nb + 127) / 128;
+        for (int ch = 0; ch < nchunk && ok; ++ch) {
+          bool any = false;
+          for (int e = 0; e < 4; ++e) {
+            const int wd = 4 * ch + e;
+            if (wd >= p.Nw) break;
+            const int jb = 32 * wd;
+            const int nvalid = min(32, p.Nb - jb);
+            const uint32_t valid = nvalid >= 32 ? 0xffffffffu : ((1u << nvalid) - 1u);
+            if ((~row0[wd] & valid) || (has_hi && (~row1[wd] & valid))) any = true;
+          }
+          if (any) push(TileDesc{kTilePooled, ch, ch, 0});
+        }
+      }
+      if (have_prev && ok) {
+        prev.flags |= 0x100u;
+        issue(prev);
+      }
+      if (!ok) set_timeout(p.status);
+      // never leave the CTA with bulk copies in flight
+      for (int u = max(0, t - kStages); u < t; ++u) mbar_wait(&sm.full[u % kStages], (u / kStages) & 1, abort);
+      mbar_wait(&sm.qfull, 0, abort);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&sm.qfull, 0, abort);
+      const uint32_t q_base = smem_u32(&sm.q[0][0]);
+      const uint32_t p_base = smem_u32(&sm.p[0][0]);
+      uint32_t prev_kind = kTilePair;
+      auto issue_pv = [&](int u, uint32_t kind) {
+        if (!mbar_wait(&sm.pready, u & 1, abort)) return false;
+        tc_fence_after();
+        const int s = u % kStages;
+        const int nsteps = kind == kTileSingle ? 4 : 8;
+        const uint32_t idesc = idesc_bf16(128, 128, false, true);
+        const uint32_t v_base = smem_u32(&sm.v[s][0][0]);
+        for (int kk = 0; kk < nsteps; ++kk) {
+          const uint64_t ad = sdesc_sw128(p_base + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(v_base + kk * 2048, kTileBytes, 1024);
+          umma_ss(tmem + 256, ad, bd, idesc, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&sm.empty[s]);
+        umma_commit(&sm.pvdone);
+        return true;
+      };
+      for (int t = 0; ok; ++t) {
+        const int s = t % kStages;
+        if (!mbar_wait(&sm.full[s], (t / kStages) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        const TileDesc d = sm.desc[s];
+        const int bsel = t & 1;
+        if (t >= 2 && !mbar_wait(&sm.sfree[bsel], ((t >> 1) - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int n = d.kind == kTileSingle ? 64 : 128;
+        const uint32_t idesc = idesc_bf16(128, n, false, false);
+        const uint32_t k_base = smem_u32(&sm.k[s][0][0]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kTileBytes + (kk & 3) * 32;
+          umma_ss(tmem + 128 * bsel, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
+                  idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.sfull[bsel]);
+        if (t > 0 && !issue_pv(t - 1, prev_kind)) {
+          ok = false;
+          break;
+        }
+        prev_kind = d.kind;
+        if (d.flags & 0x100u) {
+          ok = issue_pv(t, d.kind);
+          break;
+        }
+      }
+      if (!ok) set_timeout(p.status);
+      umma_commit(&sm.mmadone);
+      mbar_wait(&sm.mmadone, 0, abort);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // --------------------------------------------------------------- softmax / correction / epilogue
+    const int r = tid - 128;                  // query row within the tile == TMEM lane
+    const int hf = r >> 6;
+    const int qi = qb0 + hf;
+    const int tok = 64 * qb0 + r;
+    const bool row_valid = tok < p.N;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
+    const uint32_t* mrow = p.mask + ((size_t)bh * p.Nb + min(qi, p.Nb - 1)) * p.Nw;
+    const float sc = kScale * kLog2e;
+    const int n_last = p.N - 64 * (p.Nb - 1);
+    const float lg_last = log2f((float)n_last);
+    const uint32_t p_row = smem_u32(&sm.p[0][0]) + (r >> 3) * 1024 + (r & 7) * 128;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    int t = 0;
+    for (;; ++t) {
+      const int bsel = t & 1;
+      const int s = t % kStages;
+      if (!mbar_wait(&sm.sfull[bsel], (t >> 1) & 1, abort) || !mbar_wait(&sm.full[s], (t / kStages) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      const TileDesc d = sm.desc[s];
+      tc_fence_after();
+      float x[128];
+      {
+        uint32_t raw[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          if (c4 < 2 || d.kind != kTileSingle) {
+            tmem_ld32(lane_addr + 128 * bsel + 32 * c4, raw);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[32 * c4 + e] = __uint_as_float(raw[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[32 * c4 + e] = -INFINITY;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.sfree[bsel]);
+
+      // scale, bias and mask the 128 columns
+      if (d.kind == kTilePooled) {
+        uint32_t mw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int wd = 4 * d.j0 + e;
+          mw[e] = wd < p.Nw ? mrow[wd] : 0xffffffffu;
+        }
+        const int jbase = 128 * d.j0;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int j = jbase + c;
+          const bool exact = (mw[c >> 5] >> (c & 31)) & 1u;
+          const float bias = (j == p.Nb - 1) ? lg_last : 6.0f;
+          x[c] = (j < p.Nb && !exact) ? fmaf(x[c], sc, bias) : -INFINITY;
+        }
+      } else {
+        const bool v0 = (d.flags >> hf) & 1u;
+        const bool v1 = (d.kind == kTilePair) && ((d.flags >> (2 + hf)) & 1u);
+        const int lim0 = v0 ? p.N - 64 * d.j0 : 0;
+        const int lim1 = v1 ? p.N - 64 * d.j1 : 0;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = c < lim0 ? x[c] * sc : -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[64 + c] = c < lim1 ? x[64 + c] * sc : -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m_ref, mx);
+      const bool upd = m_new > m_ref + 8.0f;
+      const float m_use = upd ? m_new : m_ref;
+      const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+      const float alpha = upd ? ex2(m_ref - m_sub) : 1.f;
+      float rs = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2(x[2 * c] - m_sub);
+        const float p1 = ex2(x[2 * c + 1] - m_sub);
+        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + rs;
+      // P buffer and O are free once the previous tile's P V has completed
+      if (t > 0 && !mbar_wait(&sm.pvdone, (t - 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // tcgen05.ld / st are warp-collective: the warp rescales if any of its rows needs it
+      const bool need = upd && t > 0 && m_ref != -INFINITY;
+      if (__any_sync(0xffffffffu, need)) {
+        const float f = need ? alpha : 1.f;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + 256 + 32 * c4, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+          tmem_st32(lane_addr + 256 + 32 * c4, o);
+        }
+        tmem_st_wait();
+      }
+      m_ref = m_use;
+      // P row -> shared memory, 128-byte swizzled K-major layout (16-byte chunk index ^ row % 8)
+#pragma unroll
+      for (int c8 = 0; c8 < 16; ++c8) {
+        const uint32_t addr = p_row + (c8 >> 3) * kTileBytes + ((((uint32_t)c8 & 7u) ^ ((uint32_t)r & 7u)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c8]), "r"(pk[4 * c8 + 1]),
+                     "r"(pk[4 * c8 + 2]), "r"(pk[4 * c8 + 3])
+                     : "memory");
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.pready);
+      if (d.flags & 0x100u) break;
+    }
+    if (ok && !mbar_wait(&sm.pvdone, t & 1, abort)) ok = false;
+    if (!ok) set_timeout(p.status);
+    tc_fence_after();
+    if (__all_sync(0xffffffffu, ok)) {
+      // epilogue: o = O / l (Sol-Attn2: merged with the anchor's complementary tail)
+      float scale_o = 1.f / l;
+      float tail_w = 0.f;
+      const float* nu = nullptr;
+      if (kSol2 && row_valid) {
+        const int a = tok / 32;
+        const size_t abase = (size_t)bh * p.Na + a;
+        const float logz = p.tail_logz[abase];
+        if (logz != -INFINITY) {
+          const float* mu = p.tail_mu + abase * 128;
+          const float* qa = p.qanchor + abase * 128;
+          float delta = 0.f;
+          const uint32_t q_row = smem_u32(&sm.q[0][0]) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll 4
+          for (int c8 = 0; c8 < 16; ++c8) {
+            const uint32_t addr = q_row + (c8 >> 3) * kTileBytes + ((((uint32_t)c8 & 7u) ^ ((uint32_t)r & 7u)) << 4);
+            uint32_t w4[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
+                         : "r"(addr));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+              const int dd = 8 * c8 + 2 * e;
+              delta = fmaf(f.x - qa[dd], mu[dd], delta);
+              delta = fmaf(f.y - qa[dd + 1], mu[dd + 1], delta);
+            }
+          }
+          const float lz2 = (logz + kScale * delta) * kLog2e;  // log2 of Zhat_i
+          const float M = fmaxf(m_ref, lz2);
+          const float eo = ex2(m_ref - M);
+          tail_w = ex2(lz2 - M);
+          const float den = l * eo + tail_w;
+          scale_o = eo / den;
+          tail_w = tail_w / den;
+          nu = p.tail_nu + abase * 128;
+        }
+      }
+      {
+        __nv_bfloat16* orow = p.out + ((size_t)((size_t)b * p.N + min(tok, p.N - 1)) * p.H + h) * 128;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + 256 + 32 * c4, o);   // warp-collective: every lane loads
+          tmem_ld_wait();
+          if (!row_valid) continue;
+          uint32_t packed[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float a0 = __uint_as_float(o[2 * e]) * scale_o;
+            float a1 = __uint_as_float(o[2 * e + 1]) * scale_o;
+            if (kSol2 && nu) {
+              a0 = fmaf(tail_w, nu[32 * c4 + 2 * e], a0);
+              a1 = fmaf(tail_w, nu[32 * c4 + 2 * e + 1], a1);
+            }
+            packed[e] = pack_bf16x2(a0, a1);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * e) =
+                make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+size_t attn_fwd_smem_bytes() { return kSmemBytes; }
+
+template <bool kSol2>
+static cudaError_t launch_impl(const CUtensorMap* maps, const FwdParams& p, int units, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<kSol2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  attn_fwd_kernel<kSol2><<<units, 256, kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd(const CUtensorMap* maps, const FwdParams& p, int units, bool sol2, cudaStream_t st) {
+  return sol2 ? launch_impl<true>(maps, p, units, st) : launch_impl<false>(maps, p, units, st);
+}
+
+}  // namespace sol

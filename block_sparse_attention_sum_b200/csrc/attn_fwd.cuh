@@ -1,0 +1,28 @@
+// Launch interface of the fused attention kernel.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace sol {
+
+struct FwdParams {
+  int N, H, Nb, Nw, Na, QT;
+  const uint32_t* mask;      // [BH][Nb][Nw]
+  const int* order;          // unit order (nullptr: identity)
+  __nv_bfloat16* out;        // [B][N][H][128]
+  int* status;               // device status word
+  // Sol-Attn2 tail (unused by Sol-Attn)
+  const float* qanchor;      // [BH][Na][128]
+  const float* tail_logz;    // [BH][Na]
+  const float* tail_mu;      // [BH][Na][128]
+  const float* tail_nu;      // [BH][Na][128]
+};
+
+// maps: q, k, v (4-D over BTHD, box 64 channels x 1 head x 64 tokens x 1 batch) and the pooled
+// key / value means (3-D over [BH][Nb][128], box 64 channels x 128 blocks x 1).
+cudaError_t launch_attn_fwd(const CUtensorMap* maps, const FwdParams& p, int units, bool sol2, cudaStream_t st);
+size_t attn_fwd_smem_bytes();
+
+}  // namespace sol

@@ -1,0 +1,73 @@
+// Shapes, workspace layout and kernel declarations shared by the host launcher and the kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace sol {
+
+constexpr int kHeadDim = 128;   // head dimension (fixed by the operator's contract)
+constexpr int kBlock = 64;      // query / key block size (64 x 64 physical blocks)
+constexpr int kAnchor = 32;     // Sol-Attn2 query anchor size
+constexpr float kScale = 0.088388347648318440550f;        // 1 / sqrt(128)
+constexpr float kLog2e = 1.4426950408889634074f;
+
+struct Shape {
+  int B, N, H;
+  int Nb;   // key / query blocks
+  int Nw;   // 32-bit words per bitmask row
+  int Na;   // Sol-Attn2 anchors
+  int BH;
+  int QT;   // 128-row query tiles (pairs of query blocks)
+};
+
+inline Shape make_shape(int B, int N, int H) {
+  Shape s;
+  s.B = B;
+  s.N = N;
+  s.H = H;
+  s.Nb = (N + kBlock - 1) / kBlock;
+  s.Nw = (s.Nb + 31) / 32;
+  s.Na = (N + kAnchor - 1) / kAnchor;
+  s.BH = B * H;
+  s.QT = (s.Nb + 1) / 2;
+  return s;
+}
+
+// Device buffers of one call (all inside the library workspace).
+struct Work {
+  float* qbar;            // [BH][Nb][128]  block means of Q
+  float* kbar;            // [BH][Nb][128]  block means of K
+  __nv_bfloat16* kbar_h;  // [BH][Nb][128]  BF16 copy of kbar (surrogate MMA operand)
+  __nv_bfloat16* vbar_h;  // [BH][Nb][128]  BF16 block means of V (surrogate MMA operand)
+  float* kcov;            // [BH][128][128] centred covariance of the key-block means
+  double* kmean;          // [BH][128]      mean of the key-block means
+  float* thresh;          // [BH][Nb]       tau_i
+  uint32_t* mask;         // [BH][Nb][Nw]   exact-block bitmask
+  int* rowcount;          // [BH][Nb]       exact blocks per query-block row
+  unsigned long long* stats;  // [0] exact pairs, [1] min row, [2] max row (as unsigned)
+  // Sol-Attn2
+  float* qanchor;         // [BH][Na][128]  anchor means of Q
+  float* qdir;            // [BH][128]      mean query (the grouping direction)
+  float* gk;              // [BH][Nb][2][128] group key means
+  float* gv;              // [BH][Nb][2][128] group value means
+  int* gcount;            // [BH][Nb][2]    group sizes
+  float* tail_logz;       // [BH][Na]       log Z_a (-inf for an empty tail)
+  float* tail_mu;         // [BH][Na][128]
+  float* tail_nu;         // [BH][Na][128]
+};
+
+// Prep kernels (summary.cu)
+void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
+                    const Work& w, bool anchors, cudaStream_t st);
+void launch_kstats(const Shape& s, const Work& w, cudaStream_t st);
+void launch_thresh(const Shape& s, const Work& w, float tau, cudaStream_t st);
+void launch_route(const Shape& s, const Work& w, int sink_b0, int sink_b1, cudaStream_t st);
+void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, cudaStream_t st);
+
+// Sol-Attn2 prep (sol2_tail.cu)
+void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
+                   const Work& w, cudaStream_t st);
+void launch_anchor_tail(const Shape& s, const Work& w, cudaStream_t st);
+
+}  // namespace sol

@@ -1,0 +1,190 @@
+"""Python binding of the C ABI in include/sol_attn.h (argument marshalling only).
+
+Every step of the operator runs in the CUDA library ``libsolattn.so`` built in this directory; there
+is no fallback.  If the library is missing, every call raises.  PyTorch provides device memory and
+streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+HEAD_DIM = 128
+BLOCK = 64
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
+
+# include/sol_attn.h, in declaration order
+EXPORTS = [
+    "sol_attn_fwd",
+    "sol_attn2_fwd",
+    "sol_attn_last_error",
+    "sol_attn_get_device_status",
+    "sol_attn_debug_route",
+    "sol_attn_last_stats",
+    "sol_attn_set_kernel_timing",
+    "sol_attn_last_kernel_ms",
+    "sol_attn_kernel_ms_sum",
+    "sol_attn_last_launch_count",
+    "sol_attn_release_workspace",
+]
+
+STATUS = {
+    0: "SOL_OK", -1: "SOL_ERR_NULL", -2: "SOL_ERR_SHAPE", -3: "SOL_ERR_TAU", -4: "SOL_ERR_SINK",
+    -5: "SOL_ERR_ALIGN", -6: "SOL_ERR_ALLOC", -7: "SOL_ERR_LAUNCH", -8: "SOL_ERR_DEVICE", -9: "SOL_ERR_TIMEOUT",
+}
+
+
+class SolAttnError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"{STATUS.get(code, code)}: {message}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"Sol-Attn CUDA library not found at {path}; build it with "
+                           "`python -m block_sparse_attention_sum_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fwd_args = [vp, vp, vp, vp, i, i, i, f, i, i, vp]
+    lib.sol_attn_fwd.argtypes = fwd_args
+    lib.sol_attn_fwd.restype = i
+    lib.sol_attn2_fwd.argtypes = fwd_args
+    lib.sol_attn2_fwd.restype = i
+    lib.sol_attn_last_error.argtypes = []
+    lib.sol_attn_last_error.restype = ctypes.c_char_p
+    lib.sol_attn_get_device_status.argtypes = [vp]
+    lib.sol_attn_get_device_status.restype = i
+    lib.sol_attn_debug_route.argtypes = [vp, vp, i, i, i, f, i, i, vp, vp, vp]
+    lib.sol_attn_debug_route.restype = i
+    ll = ctypes.POINTER(ctypes.c_longlong)
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.sol_attn_last_stats.argtypes = [ll, ll, ip, ip]
+    lib.sol_attn_last_stats.restype = i
+    lib.sol_attn_set_kernel_timing.argtypes = [i]
+    lib.sol_attn_set_kernel_timing.restype = i
+    lib.sol_attn_last_kernel_ms.argtypes = []
+    lib.sol_attn_last_kernel_ms.restype = f
+    lib.sol_attn_kernel_ms_sum.argtypes = [i]
+    lib.sol_attn_kernel_ms_sum.restype = f
+    lib.sol_attn_last_launch_count.argtypes = []
+    lib.sol_attn_last_launch_count.restype = i
+    lib.sol_attn_release_workspace.argtypes = []
+    lib.sol_attn_release_workspace.restype = None
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        msg = load_library().sol_attn_last_error().decode(errors="replace")
+        raise SolAttnError(rc, msg)
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_qkv(q, k, v=None):
+    ts = [q, k] if v is None else [q, k, v]
+    for t in ts:
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError("q, k, v must be CUDA tensors")
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or t.shape[-1] != HEAD_DIM or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous BF16 [B, N, H, 128] (BTHD)")
+        if t.shape != q.shape or t.device != q.device:
+            raise ValueError("q, k, v must share shape and device")
+    return q.shape[0], q.shape[1], q.shape[2]
+
+
+def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream):
+    B, N, H = _check_qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device != q.device:
+        raise ValueError("out must be a contiguous BF16 tensor shaped like q")
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = getattr(lib, fn_name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H,
+                                   float(tau), int(sink_start), int(sink_tokens), _stream_handle(stream))
+    _check(rc)
+    return out
+
+
+def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
+    """Sol-Attn forward through the C ABI; returns ``out`` (BF16 [B, N, H, 128])."""
+    return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream)
+
+
+def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
+    """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
+    return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream)
+
+
+def sol_attn(q, k, v, tau=1.0, sink_start=None, sink_tokens=0, out=None):
+    """README-style entry: ``sink_start=None`` with ``sink_tokens > 0`` selects a suffix sink."""
+    return sol_attn_fwd(q, k, v, tau, -1 if sink_start is None else sink_start, sink_tokens, out)
+
+
+def sol_attn2(q, k, v, tau=1.0, sink_start=None, sink_tokens=0, out=None):
+    return sol_attn2_fwd(q, k, v, tau, -1 if sink_start is None else sink_start, sink_tokens, out)
+
+
+def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None):
+    """Exact-block mask (uint8 [B, H, Nb, Nb]) and thresholds (float32 [B, H, Nb]) from the GPU router."""
+    B, N, H = _check_qkv(q, k)
+    Nb = math.ceil(N / BLOCK)
+    mask = torch.empty(B, H, Nb, Nb, dtype=torch.uint8, device=q.device)
+    thresh = torch.empty(B, H, Nb, dtype=torch.float32, device=q.device)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.sol_attn_debug_route(q.data_ptr(), k.data_ptr(), B, N, H, float(tau), int(sink_start),
+                                      int(sink_tokens), mask.data_ptr(), thresh.data_ptr(), _stream_handle(stream))
+    _check(rc)
+    return mask, thresh
+
+
+def last_stats():
+    """(exact_pairs, total_pairs, min_row, max_row) of the most recent call on its device."""
+    lib = load_library()
+    e, t = ctypes.c_longlong(), ctypes.c_longlong()
+    mn, mx = ctypes.c_int(), ctypes.c_int()
+    _check(lib.sol_attn_last_stats(ctypes.byref(e), ctypes.byref(t), ctypes.byref(mn), ctypes.byref(mx)))
+    return e.value, t.value, mn.value, mx.value
+
+
+def get_device_status(stream=None) -> int:
+    return load_library().sol_attn_get_device_status(_stream_handle(stream))
+
+
+def set_kernel_timing(enable: bool):
+    _check(load_library().sol_attn_set_kernel_timing(1 if enable else 0))
+
+
+def last_kernel_ms() -> float:
+    return float(load_library().sol_attn_last_kernel_ms())
+
+
+def kernel_ms_sum(n: int) -> float:
+    """Summed fused-kernel duration (ms) of the last n timed launches."""
+    return float(load_library().sol_attn_kernel_ms_sum(int(n)))
+
+
+def last_launch_count() -> int:
+    return int(load_library().sol_attn_last_launch_count())
+
+
+def release_workspace():
+    load_library().sol_attn_release_workspace()

@@ -1,0 +1,133 @@
+/*
+ * sol_attn.h -- C ABI of the B200 (sm_100a) Sol-Attn / Sol-Attn2 forward library.
+ *
+ * Operation (what the entry points compute), from the pages:
+ *   "Sol-Attn: Accelerating Video Generation Inference via On-the-Fly Attention Sparsification"
+ *   (arXiv 2607.24027): section 3.1 (query-dependent threshold, Eqs. (4)-(5)), section 3.2
+ *   (chunk-wise on-the-fly thresholding, proxy-score reuse as approximate correction,
+ *   hardware-aligned nested-loop kernel, Fig. 4); the Sol-Attn README (NVlabs/Sana
+ *   sparse_backends), "Core API" and "Exact KV sink"; the stable-diffusion.cpp Sol-Attn
+ *   documentation (adjacent blocks remain exact, K means and V sums); and
+ *   "Sol-Attn2: Sparse Attention with Complementary Approximation", Method, "Routing and
+ *   complementary approximation".
+ *
+ * Common conventions for every entry point
+ *   - q, k, v, out: DEVICE pointers to contiguous BF16 tensors in BTHD layout [B, N, H, 128]:
+ *     element (b, t, h, c) sits at ((b*N + t)*H + h)*128 + c.  Head dimension is fixed at 128,
+ *     attention is non-causal and unmasked, Q/K/V share N and H (self-attention).  Pointers must
+ *     be 16-byte aligned; `out` must not overlap q, k or v.  The caller owns all four buffers.
+ *   - Blocks: 64-token key/query blocks, Nb = ceil(N / 64); the last block may be partial.
+ *   - tau: the threshold coefficient beta of tau_i = mu_i + beta * sigma_i (higher selects fewer
+ *     blocks).  Must be finite; 0 does not mean dense.
+ *   - Sink: sink_tokens <= 0 means no sink.  sink_start >= 0 makes [sink_start,
+ *     sink_start + sink_tokens) exact (clipped to N); sink_start < 0 makes the suffix
+ *     [N - sink_tokens, N) exact.  sink_start >= N is an error.  Every key block overlapping the
+ *     range is exact for every query.
+ *   - stream: a cudaStream_t passed as void*.  NULL is the legacy default stream.  All work is
+ *     enqueued on it; the call returns after enqueueing (no host synchronisation), except that a
+ *     call may synchronise the device once to grow the library's workspace.
+ *   - Workspace: the library owns a per-device workspace that grows on demand and is reused.
+ *     Calls on different streams of the same device are ordered by the library (each call waits
+ *     for the previous one through an event), so they never race on the workspace.
+ *   - Return value: SOL_OK (0) or a negative sol_status.  Argument errors are detected on the host
+ *     before anything is launched.  sol_attn_last_error() gives a message for the calling thread.
+ *   - Device-side faults never trap: every wait inside a kernel is bounded (about one second)
+ *     and a wait that runs out records SOL_ERR_TIMEOUT in a device status word that
+ *     sol_attn_get_device_status() reads.
+ */
+#ifndef SOL_ATTN_H_
+#define SOL_ATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SOL_OK = 0,
+  SOL_ERR_NULL = -1,    /* a required pointer is NULL */
+  SOL_ERR_SHAPE = -2,   /* B, N or H <= 0, or sizes overflow the supported range */
+  SOL_ERR_TAU = -3,     /* tau is not finite */
+  SOL_ERR_SINK = -4,    /* sink_start >= N */
+  SOL_ERR_ALIGN = -5,   /* a tensor pointer is not 16-byte aligned, or out overlaps an input */
+  SOL_ERR_ALLOC = -6,   /* workspace allocation failed */
+  SOL_ERR_LAUNCH = -7,  /* a CUDA launch or runtime call failed */
+  SOL_ERR_DEVICE = -8,  /* no usable sm_100 device */
+  SOL_ERR_TIMEOUT = -9  /* a bounded wait inside a kernel ran out (see sol_attn_get_device_status) */
+} sol_status;
+
+/*
+ * Sol-Attn forward (arXiv 2607.24027, sections 3.1-3.2).  For each (b, h) and 64-token query
+ * block i: block means Qbar_i, Kbar_j; proxies s_ij = Qbar_i . Kbar_j / sqrt(128); threshold
+ * tau_i = mu_i + tau * sigma_i with mu_i, sigma_i the mean and standard deviation of row i of the
+ * proxy map (full covariance form, Eq. (5)); key block j is exact iff s_ij > tau_i, |i - j| <= 1,
+ * or j overlaps the sink.  Each query token attends exactly to the tokens of its exact blocks and
+ * approximately to every other block through the surrogate (logit q.Kbar_j / sqrt(128), mass
+ * n_j, value sum Vhat_j); both share one softmax normaliser.  Result rounded to BF16 in `out`.
+ */
+int sol_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                 int sink_start, int sink_tokens, void* stream);
+
+/*
+ * Sol-Attn2 complementary-tail forward ("Sol-Attn2", Method, "Routing and complementary
+ * approximation").  Same exact sets E_i as sol_attn_fwd.  Each key block is split into two groups
+ * by its keys' projection on the mean-query direction u (the mean of all queries of the (b, h)):
+ * group 1 holds keys with k.u above the block mean's projection.  For each 32-token anchor a with
+ * mean query qbar_a, over the groups of the blocks outside E of its query block:
+ * w_ag = n_g exp(qbar_a . kbar_g / sqrt(128)), Z_a = sum w, (mu_a, nu_a) = sum w (kbar_g, vbar_g) / Z_a.
+ * Query i of the anchor gets Zhat_i = Z_a exp((q_i - qbar_a) . mu_a / sqrt(128)) and
+ * o_i = (sum_{E_i} e^{z} v + Zhat_i nu_a) / (sum_{E_i} e^{z} + Zhat_i).  Same arguments as
+ * sol_attn_fwd.
+ */
+int sol_attn2_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                  int sink_start, int sink_tokens, void* stream);
+
+/* Message for the last error returned on the calling thread ("" if none).  Owned by the library. */
+const char* sol_attn_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's status word.  Returns SOL_OK, or
+ * SOL_ERR_TIMEOUT if a bounded wait inside a kernel ran out since the last read, or
+ * SOL_ERR_LAUNCH if the synchronisation itself failed.
+ */
+int sol_attn_get_device_status(void* stream);
+
+/*
+ * Routing only (test and bench introspection): runs the block-summary, threshold and routing
+ * kernels of sol_attn_fwd and expands the exact-block bitmask.
+ *   mask   : DEVICE uint8 [B, H, Nb, Nb], 1 where key block j is exact for query block i.
+ *   thresh : DEVICE float [B, H, Nb] thresholds tau_i, or NULL.
+ * Same argument rules as sol_attn_fwd; q and k only.
+ */
+int sol_attn_debug_route(const void* q, const void* k, int B, int N, int H, float tau, int sink_start,
+                         int sink_tokens, unsigned char* mask, float* thresh, void* stream);
+
+/*
+ * Realised routing statistics of the most recent sol_attn_fwd / sol_attn2_fwd /
+ * sol_attn_debug_route on this device: number of exact (query-block, key-block) pairs, number of
+ * pairs in total, and the smallest and largest number of exact blocks in one query-block row.
+ * Synchronises the stream of that call.  Any output pointer may be NULL.
+ */
+int sol_attn_last_stats(long long* exact_pairs, long long* total_pairs, int* min_row, int* max_row);
+
+/*
+ * Kernel timing for measurement: when enabled (nonzero), each forward call records a pair of CUDA
+ * events on its stream around the fused attention kernel, in a ring of 256 pairs per device that
+ * enabling resets.  sol_attn_last_kernel_ms() synchronises on the most recent closing event and
+ * returns that launch's duration in milliseconds; sol_attn_kernel_ms_sum(n) returns the summed
+ * duration of the last n timed launches (n <= 256).  Both return a negative value if unavailable.
+ */
+int sol_attn_set_kernel_timing(int enable);
+float sol_attn_last_kernel_ms(void);
+float sol_attn_kernel_ms_sum(int n);
+
+/* Number of kernels the most recent forward call launched. */
+int sol_attn_last_launch_count(void);
+
+/* Frees this process's workspaces on every device (synchronises each device first). */
+void sol_attn_release_workspace(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_ATTN_H_ */

@@ -1,0 +1,52 @@
+"""Comparison helpers for the GPU-vs-oracle parity tests.
+
+Routing decisions: the GPU mask must equal the oracle's bit for bit, except for pairs whose proxy
+margin |s_ij - tau_i| is within MARGIN (scaled units); forced pairs (adjacent, sink) must always be
+set.  Outputs: compared element by element on the query blocks whose mask rows agree, within
+MAX_ABS and REL_L2.
+"""
+import numpy as np
+
+MARGIN = 1e-3
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+
+
+def check_mask(gpu_mask, ref, sink_flags=None):
+    """Returns the boolean [B, H, Nb] array of query-block rows whose masks differ."""
+    gm = np.asarray(gpu_mask).astype(bool)
+    om = ref["mask"]
+    assert gm.shape == om.shape, (gm.shape, om.shape)
+    Nb = om.shape[-1]
+    i = np.arange(Nb)
+    adjacent = np.abs(i[:, None] - i[None, :]) <= 1
+    assert gm[..., adjacent].all(), "adjacent blocks must be exact"
+    if sink_flags is not None and sink_flags.any():
+        assert gm[..., sink_flags].all(), "sink blocks must be exact"
+    diff = gm != om
+    if diff.any():
+        margin = np.abs(ref["shat"] - ref["thresh"][..., None])
+        bad = diff & (margin > MARGIN)
+        assert not bad.any(), f"{int(bad.sum())} mask mismatches outside the {MARGIN} margin"
+    return diff.any(axis=-1)
+
+
+def compare_outputs(gpu_out, ref_out, N, skip_rows=None, qblocks=None):
+    """gpu_out: BF16/float tensor [B, N, H, 128]; ref_out: FP64 oracle (NaN where not computed)."""
+    g = np.asarray(gpu_out, dtype=np.float64)
+    r = np.asarray(ref_out)
+    B, _, H, _ = r.shape
+    sel = ~np.isnan(r[..., 0])                  # [B, N, H]
+    if skip_rows is not None:
+        Nb = skip_rows.shape[-1]
+        tok_blk = np.minimum(np.arange(N) // 64, Nb - 1)
+        skip_tok = skip_rows[:, :, tok_blk].transpose(0, 2, 1)   # [B, N, H]
+        sel &= ~skip_tok
+    assert sel.any(), "nothing to compare"
+    d = g[sel] - r[sel]
+    max_abs = float(np.abs(d).max())
+    rel = float(np.linalg.norm(d) / max(np.linalg.norm(r[sel]), 1e-30))
+    assert np.isfinite(g[sel]).all(), "non-finite GPU output"
+    assert max_abs <= MAX_ABS, f"max abs error {max_abs:.3e} > {MAX_ABS}"
+    assert rel <= REL_L2, f"relative l2 error {rel:.3e} > {REL_L2}"
+    return max_abs, rel, int(sel.sum())

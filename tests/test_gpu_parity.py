@@ -1,0 +1,153 @@
+"""GPU parity: the CUDA library (through its C ABI) against the FP64 oracle on the same inputs.
+
+Routing: masks bit-exact outside the 1e-3 proxy margin, forced blocks always exact, thresholds to
+FP32 rounding.  Outputs: max-abs <= 2e-2 and relative l2 <= 5e-3 against the oracle, element by
+element, on every query block whose mask row agrees (all of them unless a near-tie flipped).
+Small and ragged shapes run in full; the 32K-128K workloads compare 16 seeded query blocks per head
+(all heads) plus the full routing mask, in the launch configuration the bench times.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_sum_b200 import sol_attn as sa
+from block_sparse_attention_sum_b200.inputs import iid_qkv
+from block_sparse_attention_sum_b200.workloads import WORKLOADS
+from oracle import sol_attn_oracle as orc
+from tests.parity import check_mask, compare_outputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _to_gpu(*ts):
+    return [t.cuda() for t in ts]
+
+
+def _run(entry, q, k, v, tau, sink_start, sink_tokens):
+    qd, kd, vd = _to_gpu(q, k, v)
+    fn = sa.sol_attn_fwd if entry == "sol_attn" else sa.sol_attn2_fwd
+    out = fn(qd, kd, vd, tau, sink_start, sink_tokens)
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    return out.float().cpu().numpy(), (qd, kd, vd)
+
+
+SMALL = [
+    # name, B, N, H, tau, sink_start, sink_tokens
+    ("n64", 1, 64, 1, 1.0, -1, 0),
+    ("n65_b2_h3", 2, 65, 3, 1.0, -1, 0),
+    ("n127", 1, 127, 2, 0.5, -1, 0),
+    ("n129", 1, 129, 2, 1.0, -1, 0),
+    ("n200_suffix_sink", 1, 200, 2, 1.0, -1, 10),
+    ("n1000_b2", 2, 1000, 2, 1.0, -1, 0),
+    ("n1000_interior_sink", 1, 1000, 2, 1.5, 300, 200),
+    ("n2048_dense_sink", 1, 2048, 2, 1.0, 0, 2048),
+    ("n4000_high_tau", 1, 4000, 2, 3.0, -1, 0),
+    ("n4096_low_tau", 1, 4096, 1, -0.5, -1, 0),
+]
+
+
+def _small_inputs(name, B, N, H):
+    return iid_qkv(B, N, H, seed=zlib.crc32(name.encode()) % 1000)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+@pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
+def test_small_and_ragged(case, entry):
+    name, B, N, H, tau, ss, st = case
+    q, k, v = _small_inputs(name, B, N, H)
+    ref = getattr(orc, entry)(q, k, v, tau, ss, st)
+    gout, (qd, kd, _) = _run(entry, q, k, v, tau, ss, st)
+    gmask, gthr = sa.debug_route(qd, kd, tau, ss, st)
+    full = orc.routing(q, k, tau, ss, st)
+    ref.update(shat=full["shat"], thresh=full["thresh"])
+    skip = check_mask(gmask.cpu().numpy(), ref, orc.sink_block_flags(N, ss, st))
+    compare_outputs(gout, ref["out"], N, skip_rows=skip)
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan"])
+@pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
+def test_named_workloads_in_full(name, entry):
+    w = WORKLOADS[name]
+    q, k, v = w.make_inputs("cpu")
+    tau = w.resolved_tau()
+    ref = getattr(orc, entry)(q, k, v, tau, w.sink_start, w.sink_tokens)
+    full = orc.routing(q, k, tau, w.sink_start, w.sink_tokens)
+    ref.update(shat=full["shat"], thresh=full["thresh"])
+    gout, (qd, kd, _) = _run(entry, q, k, v, tau, w.sink_start, w.sink_tokens)
+    gmask, gthr = sa.debug_route(qd, kd, tau, w.sink_start, w.sink_tokens)
+    skip = check_mask(gmask.cpu().numpy(), ref)
+    assert skip.mean() <= 0.01
+    np.testing.assert_allclose(gthr.cpu().numpy(), full["thresh"], rtol=1e-5, atol=2e-6)
+    compare_outputs(gout, ref["out"], w.N, skip_rows=skip)
+
+
+LARGE = ["s32k_80", "s32k_85", "s32k_90", "s64k", "s128k", "sol2_64k"]
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_large_workloads_sampled(name):
+    w = WORKLOADS[name]
+    q, k, v = w.make_inputs("cpu")
+    tau = w.resolved_tau()
+    Nb = orc.num_blocks(w.N)
+    sample = sorted(np.random.default_rng(7).choice(Nb, size=16, replace=False).tolist())
+    fn = getattr(orc, w.entry)
+    ref = fn(q, k, v, tau, w.sink_start, w.sink_tokens, qblocks=sample)
+    full = orc.routing(q, k, tau, w.sink_start, w.sink_tokens)
+    ref.update(shat=full["shat"], thresh=full["thresh"])
+    del full
+    gout, (qd, kd, _) = _run(w.entry, q, k, v, tau, w.sink_start, w.sink_tokens)
+    exact, total, mn, mx = sa.last_stats()
+    gmask, gthr = sa.debug_route(qd, kd, tau, w.sink_start, w.sink_tokens)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref, orc.sink_block_flags(w.N, w.sink_start, w.sink_tokens))
+    assert skip.mean() <= 0.01
+    assert exact == int(gm.sum()) and total == gm.size
+    assert abs((1 - exact / total) - w.target_sparsity) < 0.01
+    np.testing.assert_allclose(gthr.cpu().numpy(), ref["thresh"], rtol=1e-5, atol=2e-6)
+    compare_outputs(gout, ref["out"], w.N, skip_rows=skip)
+
+
+def test_repeated_calls_are_bitwise_identical():
+    q, k, v = _to_gpu(*iid_qkv(1, 3000, 4, seed=5))
+    a = sa.sol_attn_fwd(q, k, v, 1.0)
+    b = sa.sol_attn_fwd(q, k, v, 1.0)
+    c = sa.sol_attn2_fwd(q, k, v, 1.0)
+    d = sa.sol_attn2_fwd(q, k, v, 1.0)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(c, d)
+
+
+def test_argument_errors_are_reported_before_launch():
+    q, k, v = _to_gpu(*iid_qkv(1, 256, 2, seed=1))
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.sol_attn_fwd(q, k, v, float("nan"))
+    assert e.value.code == -3
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.sol_attn_fwd(q, k, v, 1.0, sink_start=256, sink_tokens=4)
+    assert e.value.code == -4
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.sol_attn_fwd(q, k, v, 1.0, out=q)
+    assert e.value.code == -5
+    assert sa.get_device_status() == 0
+
+
+def test_stream_and_stats_and_timing():
+    q, k, v = _to_gpu(*iid_qkv(1, 2048, 2, seed=2))
+    s = torch.cuda.Stream()
+    sa.set_kernel_timing(True)
+    with torch.cuda.stream(s):
+        out = sa.sol_attn_fwd(q, k, v, 1.0, stream=s)
+    ms = sa.last_kernel_ms()
+    sa.set_kernel_timing(False)
+    s.synchronize()
+    ref = sa.sol_attn_fwd(q, k, v, 1.0)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert ms > 0
+    exact, total, mn, mx = sa.last_stats()
+    assert total == 2 * 32 * 32 and 0 < exact <= total and 2 <= mn <= mx <= 32
+    assert sa.last_launch_count() == 5
