@@ -108,6 +108,7 @@ size_t carve(const Shape& s, bool sol2, char* base, Work* w) {
   t.kbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
   t.vbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
   t.kcov = reinterpret_cast<float*>(take(bh * d * d * 4));
+  t.gram_partial = reinterpret_cast<float*>(take(bh * 8 * d * d * 4));
   t.kmean = reinterpret_cast<double*>(take(bh * d * 8));
   t.thresh = reinterpret_cast<float*>(take(bh * nb * 4));
   t.mask = reinterpret_cast<uint32_t*>(take(bh * nb * s.Nw * 4));
@@ -231,7 +232,7 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   launch_kstats(s, ww, st);
   launch_thresh(s, ww, tau, st);
   launch_route(s, ww, sb0, sb1, st);
-  *launches += 4;
+  *launches += 6;
   d.last_total_pairs = (long long)s.BH * s.Nb * s.Nb;
   return check_launch("routing kernels");
 }
@@ -306,6 +307,9 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
 }
 
 }  // namespace
+
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
 }  // namespace sol
 
 using namespace sol;

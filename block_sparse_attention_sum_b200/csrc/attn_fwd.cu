@@ -31,9 +31,13 @@ namespace sol {
 
 namespace {
 
-constexpr int kStages = 2;
-constexpr uint32_t kTileBytes = 128 * 64 * 2;  // one 128-row x 64-column BF16 box pair half (16 KB)
+constexpr int kStages = 3;                     // K / V ring depth
+constexpr int kDescRing = 8;                   // tile descriptors in flight (producer <= 3 tiles ahead of
+                                               // the MMAs, MMAs <= 2 ahead of the softmax)
+constexpr uint32_t kTileBytes = 128 * 64 * 2;  // 128 rows x 64 BF16 columns (one swizzled half, 16 KB)
 constexpr uint32_t kBoxBytes = 64 * 64 * 2;    // one 64-row x 64-column BF16 TMA box (8 KB)
+// TMEM columns: S double buffer, O accumulator, P double buffer (BF16 pairs)
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 
 enum : uint32_t { kTilePair = 0, kTileSingle = 1, kTilePooled = 2 };
 
@@ -47,15 +51,17 @@ struct __align__(1024) FwdSmem {
   __nv_bfloat16 q[2][128 * 64];            // [d half][128 rows x 64], K-major SW128
   __nv_bfloat16 k[kStages][2][128 * 64];   // [stage][d half][128 keys x 64]
   __nv_bfloat16 v[kStages][2][128 * 64];
-  __nv_bfloat16 p[2][128 * 64];            // [key half][128 rows x 64 keys]
-  TileDesc desc[kStages];
-  uint64_t full[kStages], empty[kStages];
+  TileDesc desc[kDescRing];
+  uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
+  uint64_t dfull[kDescRing];
   uint64_t qfull, sfull[2], sfree[2], pready, pvdone, mmadone;
+  float lsum[2][128];
   uint32_t tmem_base;
   int abort;
 };
 
 constexpr size_t kSmemBytes = sizeof(FwdSmem) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -68,7 +74,7 @@ __device__ __forceinline__ void set_timeout(int* status) { atomicExch(status, kD
 }  // namespace
 
 template <bool kSol2>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
                     const __grid_constant__ CUtensorMap tm_vp, const FwdParams p) {
@@ -85,15 +91,18 @@ __global__ void __launch_bounds__(256, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.kfull[s], 1);
+      mbar_init(&sm.kempty[s], 1);
+      mbar_init(&sm.vfull[s], 1);
+      mbar_init(&sm.vempty[s], 1);
     }
+    for (int s = 0; s < kDescRing; ++s) mbar_init(&sm.dfull[s], 1);
     mbar_init(&sm.qfull, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.sfull[i], 1);
-      mbar_init(&sm.sfree[i], 128);
+      mbar_init(&sm.sfree[i], 256);
     }
-    mbar_init(&sm.pready, 128);
+    mbar_init(&sm.pready, 256);
     mbar_init(&sm.pvdone, 1);
     mbar_init(&sm.mmadone, 1);
     sm.abort = 0;
@@ -131,27 +140,38 @@ __global__ void __launch_bounds__(256, 1)
       bool have_prev = false;
       auto issue = [&](TileDesc d) {
         const int s = t % kStages;
-        if (t >= kStages && !mbar_wait(&sm.empty[s], ((t / kStages) - 1) & 1, abort)) {
+        const uint32_t ph = ((t / kStages) - 1) & 1;
+        if (t >= kStages && !mbar_wait(&sm.kempty[s], ph, abort)) {
           ok = false;
           return;
         }
-        sm.desc[s] = d;
-        if (d.kind == kTilePooled) {
-          mbar_arrive_expect_tx(&sm.full[s], 4 * kTileBytes);
-          for (int dh = 0; dh < 2; ++dh) {
-            tma_load_3d(&sm.k[s][dh][0], &tm_kp, &sm.full[s], 64 * dh, 128 * d.j0, bh);
-            tma_load_3d(&sm.v[s][dh][0], &tm_vp, &sm.full[s], 64 * dh, 128 * d.j0, bh);
-          }
+        sm.desc[t % kDescRing] = d;
+        mbar_arrive(&sm.dfull[t % kDescRing]);
+        const bool pooled = d.kind == kTilePooled;
+        const int nblk = d.kind == kTilePair ? 2 : 1;
+        const uint32_t bytes = pooled ? 2 * kTileBytes : 2 * kBoxBytes * nblk;
+        mbar_arrive_expect_tx(&sm.kfull[s], bytes);
+        if (pooled) {
+          for (int dh = 0; dh < 2; ++dh) tma_load_3d(&sm.k[s][dh][0], &tm_kp, &sm.kfull[s], 64 * dh, 128 * d.j0, bh);
         } else {
-          const int nblk = d.kind == kTilePair ? 2 : 1;
-          mbar_arrive_expect_tx(&sm.full[s], 4 * kBoxBytes * nblk);
-          for (int slot = 0; slot < nblk; ++slot) {
-            const int j = slot ? d.j1 : d.j0;
-            for (int dh = 0; dh < 2; ++dh) {
-              tma_load_4d(&sm.k[s][dh][slot * 64 * 64], &tm_k, &sm.full[s], 64 * dh, h, 64 * j, b);
-              tma_load_4d(&sm.v[s][dh][slot * 64 * 64], &tm_v, &sm.full[s], 64 * dh, h, 64 * j, b);
-            }
-          }
+          for (int slot = 0; slot < nblk; ++slot)
+            for (int dh = 0; dh < 2; ++dh)
+              tma_load_4d(&sm.k[s][dh][slot * 64 * 64], &tm_k, &sm.kfull[s], 64 * dh, h, 64 * (slot ? d.j1 : d.j0),
+                          b);
+        }
+        if (t >= kStages && !mbar_wait(&sm.vempty[s], ph, abort)) {
+          ok = false;
+          ++t;   // the K copy of this tile is in flight
+          return;
+        }
+        mbar_arrive_expect_tx(&sm.vfull[s], bytes);
+        if (pooled) {
+          for (int dh = 0; dh < 2; ++dh) tma_load_3d(&sm.v[s][dh][0], &tm_vp, &sm.vfull[s], 64 * dh, 128 * d.j0, bh);
+        } else {
+          for (int slot = 0; slot < nblk; ++slot)
+            for (int dh = 0; dh < 2; ++dh)
+              tma_load_4d(&sm.v[s][dh][slot * 64 * 64], &tm_v, &sm.vfull[s], 64 * dh, h, 64 * (slot ? d.j1 : d.j0),
+                          b);
         }
         ++t;
       };
@@ -204,7 +224,10 @@ __global__ void __launch_bounds__(256, 1)
       }
       if (!ok) set_timeout(p.status);
       // never leave the CTA with bulk copies in flight
-      for (int u = max(0, t - kStages); u < t; ++u) mbar_wait(&sm.full[u % kStages], (u / kStages) & 1, abort);
+      for (int u = max(0, t - kStages); u < t; ++u) {
+        mbar_wait(&sm.kfull[u % kStages], (u / kStages) & 1, abort);
+        mbar_wait(&sm.vfull[u % kStages], (u / kStages) & 1, abort);
+      }
       mbar_wait(&sm.qfull, 0, abort);
     }
     __syncwarp();
@@ -213,31 +236,30 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qfull, 0, abort);
       const uint32_t q_base = smem_u32(&sm.q[0][0]);
-      const uint32_t p_base = smem_u32(&sm.p[0][0]);
       uint32_t prev_kind = kTilePair;
       auto issue_pv = [&](int u, uint32_t kind) {
-        if (!mbar_wait(&sm.pready, u & 1, abort)) return false;
-        tc_fence_after();
         const int s = u % kStages;
+        if (!mbar_wait(&sm.pready, u & 1, abort) || !mbar_wait(&sm.vfull[s], (u / kStages) & 1, abort)) return false;
+        tc_fence_after();
         const int nsteps = kind == kTileSingle ? 4 : 8;
         const uint32_t idesc = idesc_bf16(128, 128, false, true);
         const uint32_t v_base = smem_u32(&sm.v[s][0][0]);
+        const uint32_t p_col = tmem + kColP + 64 * (u & 1);
         for (int kk = 0; kk < nsteps; ++kk) {
-          const uint64_t ad = sdesc_sw128(p_base + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(v_base + kk * 2048, kTileBytes, 1024);
-          umma_ss(tmem + 256, ad, bd, idesc, (u > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + kColO, p_col + 8 * kk, bd, idesc, (u > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&sm.empty[s]);
+        umma_commit(&sm.vempty[s]);
         umma_commit(&sm.pvdone);
         return true;
       };
       for (int t = 0; ok; ++t) {
         const int s = t % kStages;
-        if (!mbar_wait(&sm.full[s], (t / kStages) & 1, abort)) {
+        if (!mbar_wait(&sm.kfull[s], (t / kStages) & 1, abort)) {
           ok = false;
           break;
         }
-        const TileDesc d = sm.desc[s];
+        const TileDesc d = sm.desc[t % kDescRing];
         const int bsel = t & 1;
         if (t >= 2 && !mbar_wait(&sm.sfree[bsel], ((t >> 1) - 1) & 1, abort)) {
           ok = false;
@@ -249,10 +271,11 @@ __global__ void __launch_bounds__(256, 1)
         const uint32_t k_base = smem_u32(&sm.k[s][0][0]);
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kTileBytes + (kk & 3) * 32;
-          umma_ss(tmem + 128 * bsel, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
-                  idesc, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + kColS + 128 * bsel, sdesc_sw128(q_base + off, 16, 1024),
+                  sdesc_sw128(k_base + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sm.sfull[bsel]);
+        umma_commit(&sm.kempty[s]);
         if (t > 0 && !issue_pv(t - 1, prev_kind)) {
           ok = false;
           break;
@@ -270,49 +293,49 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // --------------------------------------------------------------- softmax / correction / epilogue
-    const int r = tid - 128;                  // query row within the tile == TMEM lane
+    // Two warpgroups share the 128 rows (TMEM lane = row); warpgroup wg owns columns 64 wg .. 64 wg + 63
+    // of S, P and O.  Both compute the full row max (so they agree on the reference max without
+    // exchanging it) and exponentiate only their own half; their partial row sums are added at the end.
+    const int wg = (warp - 4) >> 2;
+    const int r = ((warp & 3) << 5) | lane;   // query row within the tile == TMEM lane
     const int hf = r >> 6;
     const int qi = qb0 + hf;
     const int tok = 64 * qb0 + r;
     const bool row_valid = tok < p.N;
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t* mrow = p.mask + ((size_t)bh * p.Nb + min(qi, p.Nb - 1)) * p.Nw;
     const float sc = kScale * kLog2e;
     const int n_last = p.N - 64 * (p.Nb - 1);
     const float lg_last = log2f((float)n_last);
-    const uint32_t p_row = smem_u32(&sm.p[0][0]) + (r >> 3) * 1024 + (r & 7) * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     int t = 0;
     for (;; ++t) {
       const int bsel = t & 1;
-      const int s = t % kStages;
-      if (!mbar_wait(&sm.sfull[bsel], (t >> 1) & 1, abort) || !mbar_wait(&sm.full[s], (t / kStages) & 1, abort)) {
+      if (!mbar_wait(&sm.dfull[t % kDescRing], (t / kDescRing) & 1, abort) ||
+          !mbar_wait(&sm.sfull[bsel], (t >> 1) & 1, abort)) {
         ok = false;
         break;
       }
-      const TileDesc d = sm.desc[s];
+      const TileDesc d = sm.desc[t % kDescRing];
       tc_fence_after();
-      float x[128];
-      {
-        uint32_t raw[32];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          if (c4 < 2 || d.kind != kTileSingle) {
-            tmem_ld32(lane_addr + 128 * bsel + 32 * c4, raw);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[32 * c4 + e] = __uint_as_float(raw[e]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[32 * c4 + e] = -INFINITY;
-          }
-        }
+      const bool single = d.kind == kTileSingle;
+      uint32_t own[64], oth[32];
+      const uint32_t s_addr = lane_addr + kColS + 128 * bsel;
+      const uint32_t oth_addr = s_addr + 64 * (1 - wg);
+      const bool have_own = !single || wg == 0, have_oth = !single || wg == 1;
+      if (have_own) {
+        tmem_ld32_at<0>(s_addr + 64 * wg, own);
+        tmem_ld32_at<32>(s_addr + 64 * wg + 32, own);
       }
-      tc_fence_before();
-      mbar_arrive(&sm.sfree[bsel]);
 
-      // scale, bias and mask the 128 columns
+      // x: own columns (in place over the raw scores); the other half only feeds the row max.
+      // Exact tiles keep raw scores (the scale is folded into the exponent), pooled tiles carry
+      // scale and log2(n_j) bias.
+      float* x = reinterpret_cast<float*>(own);
+      float mp[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mp[k] = -INFINITY;
       if (d.kind == kTilePooled) {
         uint32_t mw[4];
 #pragma unroll
@@ -320,73 +343,107 @@ __global__ void __launch_bounds__(256, 1)
           const int wd = 4 * d.j0 + e;
           mw[e] = wd < p.Nw ? mrow[wd] : 0xffffffffu;
         }
-        const int jbase = 128 * d.j0;
+        const int jb_own = 128 * d.j0 + 64 * wg, jb_oth = 128 * d.j0 + 64 * (1 - wg);
+        const uint32_t m_own0 = wg ? mw[2] : mw[0], m_own1 = wg ? mw[3] : mw[1];
+        const uint32_t m_oth0 = wg ? mw[0] : mw[2], m_oth1 = wg ? mw[1] : mw[3];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int j = jbase + c;
-          const bool exact = (mw[c >> 5] >> (c & 31)) & 1u;
+        for (int half = 0; half < 2; ++half) {
+          tmem_ld32_at<0>(oth_addr + 32 * half, oth);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int jo = jb_oth + 32 * half + c;
+            const float bo = (jo == p.Nb - 1) ? lg_last : 6.0f;
+            const bool ex = ((half ? m_oth1 : m_oth0) >> c) & 1u;
+            const float yv = (jo < p.Nb && !ex) ? fmaf(__uint_as_float(oth[c]), sc, bo) : -INFINITY;
+            mp[c & 7] = fmaxf(mp[c & 7], yv);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.sfree[bsel]);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int j = jb_own + c;
           const float bias = (j == p.Nb - 1) ? lg_last : 6.0f;
-          x[c] = (j < p.Nb && !exact) ? fmaf(x[c], sc, bias) : -INFINITY;
+          const bool ex = (((c < 32) ? m_own0 : m_own1) >> (c & 31)) & 1u;
+          x[c] = (j < p.Nb && !ex) ? fmaf(__uint_as_float(own[c]), sc, bias) : -INFINITY;
+          mp[c & 7] = fmaxf(mp[c & 7], x[c]);
         }
       } else {
+        // block of each half and whether it is exact for this row's query block
         const bool v0 = (d.flags >> hf) & 1u;
-        const bool v1 = (d.kind == kTilePair) && ((d.flags >> (2 + hf)) & 1u);
+        const bool v1 = !single && ((d.flags >> (2 + hf)) & 1u);
         const int lim0 = v0 ? p.N - 64 * d.j0 : 0;
         const int lim1 = v1 ? p.N - 64 * d.j1 : 0;
+        const int lim_own = wg ? lim1 : lim0, lim_oth = wg ? lim0 : lim1;
+        if (have_oth) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = c < lim0 ? x[c] * sc : -INFINITY;
+          for (int half = 0; half < 2; ++half) {
+            tmem_ld32_at<0>(oth_addr + 32 * half, oth);
+            tmem_ld_wait();
+            const int lim = lim_oth - 32 * half;
+            if (lim >= 32) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) x[64 + c] = c < lim1 ? x[64 + c] * sc : -INFINITY;
+              for (int c = 0; c < 32; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(oth[c]));
+            } else if (lim > 0) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) mp[c & 7] = fmaxf(mp[c & 7], c < lim ? __uint_as_float(oth[c]) : -INFINITY);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.sfree[bsel]);
+        if (lim_own < 64) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) x[c] = c < lim_own ? x[c] : -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      const bool pooled = d.kind == kTilePooled;
+      if (!pooled) mx *= sc;   // exact tiles: raw scores, base-2 scale applied here
       const float m_new = fmaxf(m_ref, mx);
       const bool upd = m_new > m_ref + 8.0f;
       const float m_use = upd ? m_new : m_ref;
       const float m_sub = m_use == -INFINITY ? 0.f : m_use;
       const float alpha = upd ? ex2(m_ref - m_sub) : 1.f;
-      float rs = 0.f;
-      uint32_t pk[64];
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
+      const float fs = pooled ? 1.f : sc;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(x[2 * c] - m_sub);
-        const float p1 = ex2(x[2 * c + 1] - m_sub);
-        rs += p0 + p1;
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2(fmaf(x[2 * c], fs, -m_sub));
+        const float p1 = ex2(fmaf(x[2 * c + 1], fs, -m_sub));
+        rs[c & 3] += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
-      l = l * alpha + rs;
-      // P buffer and O are free once the previous tile's P V has completed
+      l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      // P buffer (t & 1) was last read by P V of tile t - 2; O must be quiet before rescaling
       if (t > 0 && !mbar_wait(&sm.pvdone, (t - 1) & 1, abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      tmem_st32_at<0>(lane_addr + kColP + 64 * bsel + 32 * wg, pk);
       // tcgen05.ld / st are warp-collective: the warp rescales if any of its rows needs it
       const bool need = upd && t > 0 && m_ref != -INFINITY;
       if (__any_sync(0xffffffffu, need)) {
         const float f = need ? alpha : 1.f;
+        uint32_t o[64];
+        const uint32_t o_addr = lane_addr + kColO + 64 * wg;
+        tmem_ld32_at<0>(o_addr, o);
+        tmem_ld32_at<32>(o_addr + 32, o);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + 256 + 32 * c4, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(lane_addr + 256 + 32 * c4, o);
-        }
-        tmem_st_wait();
+        for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+        tmem_st32_at<0>(o_addr, o);
+        tmem_st32_at<32>(o_addr + 32, o);
       }
       m_ref = m_use;
-      // P row -> shared memory, 128-byte swizzled K-major layout (16-byte chunk index ^ row % 8)
-#pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        const uint32_t addr = p_row + (c8 >> 3) * kTileBytes + ((((uint32_t)c8 & 7u) ^ ((uint32_t)r & 7u)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c8]), "r"(pk[4 * c8 + 1]),
-                     "r"(pk[4 * c8 + 2]), "r"(pk[4 * c8 + 3])
-                     : "memory");
-      }
-      fence_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&sm.pready);
       if (d.flags & 0x100u) break;
@@ -394,6 +451,10 @@ __global__ void __launch_bounds__(256, 1)
     if (ok && !mbar_wait(&sm.pvdone, t & 1, abort)) ok = false;
     if (!ok) set_timeout(p.status);
     tc_fence_after();
+    // combine the two halves' row sums
+    sm.lsum[wg][r] = l;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    l = sm.lsum[0][r] + sm.lsum[1][r];
     if (__all_sync(0xffffffffu, ok)) {
       // epilogue: o = O / l (Sol-Attn2: merged with the anchor's complementary tail)
       float scale_o = 1.f / l;
@@ -430,32 +491,31 @@ __global__ void __launch_bounds__(256, 1)
           const float den = l * eo + tail_w;
           scale_o = eo / den;
           tail_w = tail_w / den;
-          nu = p.tail_nu + abase * 128;
+          nu = p.tail_nu + abase * 128 + 64 * wg;
         }
       }
-      {
-        __nv_bfloat16* orow = p.out + ((size_t)((size_t)b * p.N + min(tok, p.N - 1)) * p.H + h) * 128;
+      uint32_t o[64];
+      const uint32_t o_addr = lane_addr + kColO + 64 * wg;
+      tmem_ld32_at<0>(o_addr, o);
+      tmem_ld32_at<32>(o_addr + 32, o);
+      tmem_ld_wait();
+      if (row_valid) {
+        __nv_bfloat16* orow = p.out + ((size_t)((size_t)b * p.N + tok) * p.H + h) * 128 + 64 * wg;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + 256 + 32 * c4, o);   // warp-collective: every lane loads
-          tmem_ld_wait();
-          if (!row_valid) continue;
-          uint32_t packed[16];
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint32_t packed[4];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float a0 = __uint_as_float(o[2 * e]) * scale_o;
-            float a1 = __uint_as_float(o[2 * e + 1]) * scale_o;
+          for (int e = 0; e < 4; ++e) {
+            const int c = 8 * c8 + 2 * e;
+            float a0 = __uint_as_float(o[c]) * scale_o;
+            float a1 = __uint_as_float(o[c + 1]) * scale_o;
             if (kSol2 && nu) {
-              a0 = fmaf(tail_w, nu[32 * c4 + 2 * e], a0);
-              a1 = fmaf(tail_w, nu[32 * c4 + 2 * e + 1], a1);
+              a0 = fmaf(tail_w, nu[c], a0);
+              a1 = fmaf(tail_w, nu[c + 1], a1);
             }
             packed[e] = pack_bf16x2(a0, a1);
           }
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * e) =
-                make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+          *reinterpret_cast<uint4*>(orow + 8 * c8) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
       }
     }
@@ -472,14 +532,10 @@ size_t attn_fwd_smem_bytes() { return kSmemBytes; }
 
 template <bool kSol2>
 static cudaError_t launch_impl(const CUtensorMap* maps, const FwdParams& p, int units, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<kSol2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  attn_fwd_kernel<kSol2><<<units, 256, kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<kSol2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  attn_fwd_kernel<kSol2><<<units, 384, kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
   return cudaGetLastError();
 }
 

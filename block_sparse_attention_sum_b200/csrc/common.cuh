@@ -41,6 +41,7 @@ struct Work {
   __nv_bfloat16* kbar_h;  // [BH][Nb][128]  BF16 copy of kbar (surrogate MMA operand)
   __nv_bfloat16* vbar_h;  // [BH][Nb][128]  BF16 block means of V (surrogate MMA operand)
   float* kcov;            // [BH][128][128] centred covariance of the key-block means
+  float* gram_partial;    // [BH][8][128][128] partial Gram sums over ranges of key blocks
   double* kmean;          // [BH][128]      mean of the key-block means
   float* thresh;          // [BH][Nb]       tau_i
   uint32_t* mask;         // [BH][Nb][Nw]   exact-block bitmask
@@ -56,6 +57,9 @@ struct Work {
   float* tail_mu;         // [BH][Na][128]
   float* tail_nu;         // [BH][Na][128]
 };
+
+// Sets the calling thread's message returned by sol_attn_last_error() (api.cu).
+void set_last_error(const char* msg);
 
 // Prep kernels (summary.cu)
 void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,

@@ -133,6 +133,18 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]: A (M x K, BF16) read from tensor memory, one row per lane, two
+// K elements per 32-bit column (lower K index in the lower half).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on an mbarrier once every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -178,6 +190,38 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
       "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Same, for an array slice starting at element `off` (compile-time).
+template <int kOff, int kN>
+__device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, uint32_t (&r)[kN]) {
+  static_assert(kOff + 32 <= kN, "slice out of range");
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[kOff + 0]), "=r"(r[kOff + 1]), "=r"(r[kOff + 2]), "=r"(r[kOff + 3]), "=r"(r[kOff + 4]),
+        "=r"(r[kOff + 5]), "=r"(r[kOff + 6]), "=r"(r[kOff + 7]), "=r"(r[kOff + 8]), "=r"(r[kOff + 9]),
+        "=r"(r[kOff + 10]), "=r"(r[kOff + 11]), "=r"(r[kOff + 12]), "=r"(r[kOff + 13]), "=r"(r[kOff + 14]),
+        "=r"(r[kOff + 15]), "=r"(r[kOff + 16]), "=r"(r[kOff + 17]), "=r"(r[kOff + 18]), "=r"(r[kOff + 19]),
+        "=r"(r[kOff + 20]), "=r"(r[kOff + 21]), "=r"(r[kOff + 22]), "=r"(r[kOff + 23]), "=r"(r[kOff + 24]),
+        "=r"(r[kOff + 25]), "=r"(r[kOff + 26]), "=r"(r[kOff + 27]), "=r"(r[kOff + 28]), "=r"(r[kOff + 29]),
+        "=r"(r[kOff + 30]), "=r"(r[kOff + 31])
+      : "r"(taddr));
+}
+
+template <int kOff, int kN>
+__device__ __forceinline__ void tmem_st32_at(uint32_t taddr, const uint32_t (&r)[kN]) {
+  static_assert(kOff + 32 <= kN, "slice out of range");
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[kOff + 0]), "r"(r[kOff + 1]), "r"(r[kOff + 2]), "r"(r[kOff + 3]), "r"(r[kOff + 4]), "r"(r[kOff + 5]),
+      "r"(r[kOff + 6]), "r"(r[kOff + 7]), "r"(r[kOff + 8]), "r"(r[kOff + 9]), "r"(r[kOff + 10]), "r"(r[kOff + 11]),
+      "r"(r[kOff + 12]), "r"(r[kOff + 13]), "r"(r[kOff + 14]), "r"(r[kOff + 15]), "r"(r[kOff + 16]),
+      "r"(r[kOff + 17]), "r"(r[kOff + 18]), "r"(r[kOff + 19]), "r"(r[kOff + 20]), "r"(r[kOff + 21]),
+      "r"(r[kOff + 22]), "r"(r[kOff + 23]), "r"(r[kOff + 24]), "r"(r[kOff + 25]), "r"(r[kOff + 26]),
+      "r"(r[kOff + 27]), "r"(r[kOff + 28]), "r"(r[kOff + 29]), "r"(r[kOff + 30]), "r"(r[kOff + 31])
       : "memory");
 }
 

@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(256) groups_kernel(const __nv_bfloat16* __rest
 constexpr int kTailAnchors = 64;
 constexpr int kTailGroups = 32;
 
-__global__ void __launch_bounds__(256) anchor_tail_kernel(Shape s, Work w) {
+__global__ void __launch_bounds__(256, 1) anchor_tail_kernel(Shape s, Work w) {
   __shared__ float gk_s[kTailGroups][kHeadDim];
   __shared__ float gv_s[kTailGroups][kHeadDim];
   __shared__ float lw_s[kTailGroups];   // ln n_g, or -inf for an empty group
@@ -189,39 +189,44 @@ __global__ void __launch_bounds__(256) anchor_tail_kernel(Shape s, Work w) {
     const int j0 = g0 >> 1;
     const uint32_t word = mrow[j0 >> 5];
     const uint32_t ex16 = (word >> (j0 & 31)) & 0xffffu;   // j0 is a multiple of 16
-    float logit[kTailGroups];
+#pragma unroll 1
+    for (int g8 = 0; g8 < kTailGroups; g8 += 8) {
+      float logit[8];
 #pragma unroll
-    for (int gg = 0; gg < kTailGroups; ++gg) {
-      float part = 0.f;
+      for (int gg = 0; gg < 8; ++gg) {
+        float part = 0.f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) part = fmaf(qa[e], gk_s[gg][4 * e + sl], part);
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      const bool exact = (ex16 >> (gg >> 1)) & 1u;
-      logit[gg] = exact ? -INFINITY : fmaf(part, kScale, lw_s[gg]);
-    }
-    float mx = m;
+        for (int e = 0; e < 32; ++e) part = fmaf(qa[e], gk_s[g8 + gg][4 * e + sl], part);
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        const bool exact = (ex16 >> ((g8 + gg) >> 1)) & 1u;
+        logit[gg] = exact ? -INFINITY : fmaf(part, kScale, lw_s[g8 + gg]);
+      }
+      float mx = m;
 #pragma unroll
-    for (int gg = 0; gg < kTailGroups; ++gg) mx = fmaxf(mx, logit[gg]);
-    if (mx == -INFINITY) continue;
-    const float alpha = __expf(m - mx);
-    Z *= alpha;
+      for (int gg = 0; gg < 8; ++gg) mx = fmaxf(mx, logit[gg]);
+      if (mx == -INFINITY) continue;
+      if (mx > m) {   // new running max: rescale the accumulators
+        const float alpha = __expf(m - mx);
+        Z *= alpha;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      acck[e] *= alpha;
-      accv[e] *= alpha;
-    }
+        for (int e = 0; e < 32; ++e) {
+          acck[e] *= alpha;
+          accv[e] *= alpha;
+        }
+        m = mx;
+      }
 #pragma unroll
-    for (int gg = 0; gg < kTailGroups; ++gg) {
-      const float wgt = __expf(logit[gg] - mx);
-      Z += wgt;
+      for (int gg = 0; gg < 8; ++gg) {
+        const float wgt = __expf(logit[gg] - m);
+        Z += wgt;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        acck[e] = fmaf(wgt, gk_s[gg][4 * e + sl], acck[e]);
-        accv[e] = fmaf(wgt, gv_s[gg][4 * e + sl], accv[e]);
+        for (int e = 0; e < 32; ++e) {
+          acck[e] = fmaf(wgt, gk_s[g8 + gg][4 * e + sl], acck[e]);
+          accv[e] = fmaf(wgt, gv_s[g8 + gg][4 * e + sl], accv[e]);
+        }
       }
     }
-    m = mx;
   }
   if (!a_valid) return;
   const size_t ab = (size_t)bh * s.Na + a;

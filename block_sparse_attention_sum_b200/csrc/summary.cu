@@ -11,9 +11,9 @@
 namespace sol {
 
 // -------------------------------------------------------------------------------------------------
-// Block summaries.  One CTA per (key block j, batch b); it walks the heads.  Each 64-token block of
-// one head is 64 rows of 256 contiguous bytes; 16 threads cover a row with 16-byte loads, 16 row
-// groups cover the block, so every warp load instruction reads two full 256-byte rows.
+// Block summaries.  One CTA per (key block j, batch b, head h).  Each 64-token block of one head is
+// 64 rows of 256 contiguous bytes; 16 threads cover a row with 16-byte loads, 16 row groups cover
+// the block, so every warp load instruction reads two full 256-byte rows.
 // Outputs per (b, h, j): Qbar, Kbar (FP32 means over the valid tokens), BF16 copies of Kbar and
 // of the value mean Vbar (surrogate MMA operands), and optionally the two 32-token anchor means of Q.
 // -------------------------------------------------------------------------------------------------
@@ -22,14 +22,14 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
                                                       const __nv_bfloat16* __restrict__ v, Shape s, Work w,
                                                       int anchors) {
   __shared__ float red[8][4][kHeadDim];
-  const int j = blockIdx.x, b = blockIdx.y;
+  const int j = blockIdx.x, b = blockIdx.y / s.H, h = blockIdx.y % s.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c16 = tid & 15, rg = tid >> 4;
   const int t0 = j * kBlock;
   const int n = min(kBlock, s.N - t0);
   const int nlo = min(n, kAnchor), nhi = n - nlo;
 
-  for (int h = 0; h < s.H; ++h) {
+  {
     float qlo[8], qhi[8], ks[8], vs[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) qlo[e] = qhi[e] = ks[e] = vs[e] = 0.f;
@@ -111,97 +111,145 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
         if (nhi > 0) w.qanchor[a0 + kHeadDim] = sqhi / (float)nhi;
       }
     }
-    __syncthreads();
   }
 }
 
 // -------------------------------------------------------------------------------------------------
-// Threshold statistics (Eq. (5)), FP64 accumulation.  kmean = mean_j Kbar_j and the centred
-// covariance C = mean_j (Kbar_j - kmean)(Kbar_j - kmean)^T, so that
-// sigma_i^2 = s^2 Qbar_i C Qbar_i^T equals Eq. (5)'s second moment minus mu_i^2 without cancellation.
-// Grid (8, BH): each CTA produces 16 rows of C (and all CTAs recompute kmean, which is cheap).
+// Threshold statistics (Eq. (5)).  kmean = mean_j Kbar_j (FP64) and the centred covariance
+// C = mean_j (Kbar_j - kmean)(Kbar_j - kmean)^T, so that sigma_i^2 = s^2 Qbar_i C Qbar_i^T equals
+// Eq. (5)'s second moment minus mu_i^2 without its cancellation.  The Gram sum is split over
+// kGramSplits ranges of key blocks (FP32 partial sums, 8 x 8 outputs per thread) and the partials
+// are combined in FP64.
 // -------------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) kstats_kernel(Shape s, Work w) {
-  __shared__ double mk[kHeadDim];
-  __shared__ double xs[32][kHeadDim];
-  const int bh = blockIdx.y, tid = threadIdx.x;
+constexpr int kGramSplits = 8;
+
+__global__ void kmean_kernel(Shape s, Work w) {
+  const int bh = blockIdx.x, c = threadIdx.x;
   const float* kb = w.kbar + (size_t)bh * s.Nb * kHeadDim;
-  if (tid < kHeadDim) {
-    double acc = 0.0;
-    for (int j = 0; j < s.Nb; ++j) acc += (double)kb[(size_t)j * kHeadDim + tid];
-    mk[tid] = acc / s.Nb;
-    if (blockIdx.x == 0) w.kmean[(size_t)bh * kHeadDim + tid] = acc / s.Nb;
-  }
+  double acc = 0.0;
+  for (int j = 0; j < s.Nb; ++j) acc += (double)kb[(size_t)j * kHeadDim + c];
+  w.kmean[(size_t)bh * kHeadDim + c] = acc / s.Nb;
+}
+
+__global__ void __launch_bounds__(256) kgram_kernel(Shape s, Work w, float* partial) {
+  __shared__ __align__(16) float xs[32][kHeadDim];
+  __shared__ float mk[kHeadDim];
+  const int bh = blockIdx.y, split = blockIdx.x, tid = threadIdx.x;
+  const int ti = tid >> 4, tj = tid & 15;
+  const float* kb = w.kbar + (size_t)bh * s.Nb * kHeadDim;
+  if (tid < kHeadDim) mk[tid] = (float)w.kmean[(size_t)bh * kHeadDim + tid];
+  const int per = (s.Nb + kGramSplits - 1) / kGramSplits;
+  const int j_lo = split * per, j_hi = min(s.Nb, j_lo + per);
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
   __syncthreads();
-  const int r = 16 * blockIdx.x + (tid >> 4);
-  const int c0 = (tid & 15) * 8;
-  double acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-  for (int j0 = 0; j0 < s.Nb; j0 += 32) {
-    const int nj = min(32, s.Nb - j0);
-    for (int idx = tid; idx < nj * kHeadDim; idx += 256) {
+  for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+    const int nj = min(32, j_hi - j0);
+    for (int idx = tid; idx < 32 * kHeadDim; idx += 256) {
       const int jj = idx / kHeadDim, c = idx % kHeadDim;
-      xs[jj][c] = (double)kb[(size_t)(j0 + jj) * kHeadDim + c] - mk[c];
+      xs[jj][c] = jj < nj ? kb[(size_t)(j0 + jj) * kHeadDim + c] - mk[c] : 0.f;
     }
     __syncthreads();
-    for (int jj = 0; jj < nj; ++jj) {
-      const double xr = xs[jj][r];
+#pragma unroll 4
+    for (int jj = 0; jj < 32; ++jj) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[jj][8 * ti]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[jj][8 * ti + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&xs[jj][8 * tj]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&xs[jj][8 * tj + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += xr * xs[jj][c0 + e];
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(av[a], bv[c], acc[a][c]);
     }
     __syncthreads();
   }
-  float* cov = w.kcov + (size_t)bh * kHeadDim * kHeadDim;
+  float* out = partial + ((size_t)bh * kGramSplits + split) * kHeadDim * kHeadDim;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) cov[r * kHeadDim + c0 + e] = (float)(acc[e] / s.Nb);
+  for (int a = 0; a < 8; ++a) {
+    float4* row = reinterpret_cast<float4*>(out + (size_t)(8 * ti + a) * kHeadDim + 8 * tj);
+    row[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    row[1] = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+  }
+}
+
+__global__ void kgram_reduce_kernel(Shape s, Work w, const float* partial) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // entry of the 128 x 128 matrix
+  if (e >= kHeadDim * kHeadDim) return;
+  double acc = 0.0;
+  for (int sp = 0; sp < kGramSplits; ++sp)
+    acc += (double)partial[((size_t)bh * kGramSplits + sp) * kHeadDim * kHeadDim + e];
+  w.kcov[(size_t)bh * kHeadDim * kHeadDim + e] = (float)(acc / s.Nb);
 }
 
 // -------------------------------------------------------------------------------------------------
-// tau_i = mu_i + tau * sigma_i with mu_i = s Qbar_i . kmean, sigma_i^2 = s^2 Qbar_i C Qbar_i^T (FP64),
-// stored rounded to FP32, the precision the routing comparison is made in.
-// Grid (ceil(Nb / 64), BH), 8 warps x 8 rows.
+// tau_i = mu_i + tau * sigma_i with mu_i = s Qbar_i . kmean and sigma_i^2 = s^2 Qbar_i C Qbar_i^T,
+// stored as FP32, the precision the routing comparison is made in.  A CTA evaluates 64 rows:
+// Y = Qbar C as a 64 x 128 x 128 product (4 rows x 8 columns per thread, FP32), then the row dot
+// products Qbar_i . Y_i and Qbar_i . kmean.  Grid (ceil(Nb / 64), BH), 256 threads.
 // -------------------------------------------------------------------------------------------------
+constexpr int kThreshPad = 68;
+
 __global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau) {
-  extern __shared__ float cov_s[];  // [128][128]
-  __shared__ double qrow[8][kHeadDim];
-  const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ __align__(16) float tsm[];
+  float* cov_s = tsm;                                // [128][128]
+  float* qt = tsm + kHeadDim * kHeadDim;             // [128][68]  Qbar^T of the 64 rows
+  __shared__ float part[64][17];
+  __shared__ float mu_s[64];
+  const int bh = blockIdx.y, i0 = blockIdx.x * 64, tid = threadIdx.x;
   const float* cov = w.kcov + (size_t)bh * kHeadDim * kHeadDim;
+  const float* qb = w.qbar + (size_t)bh * s.Nb * kHeadDim;
   for (int idx = tid; idx < kHeadDim * kHeadDim / 4; idx += 256)
     reinterpret_cast<float4*>(cov_s)[idx] = reinterpret_cast<const float4*>(cov)[idx];
+  for (int idx = tid; idx < 64 * kHeadDim; idx += 256) {
+    const int r = idx / kHeadDim, c = idx % kHeadDim;
+    qt[c * kThreshPad + r] = (i0 + r < s.Nb) ? qb[(size_t)(i0 + r) * kHeadDim + c] : 0.f;
+  }
   __syncthreads();
-  const double* mk = w.kmean + (size_t)bh * kHeadDim;
-  for (int rr = 0; rr < 8; ++rr) {
-    const int i = blockIdx.x * 64 + warp * 8 + rr;
-    if (i >= s.Nb) break;
-    const float* qb = w.qbar + ((size_t)bh * s.Nb + i) * kHeadDim;
-    double mu = 0.0;
-    for (int c = lane; c < kHeadDim; c += 32) {
-      const double x = (double)qb[c];
-      qrow[warp][c] = x;
-      mu += x * mk[c];
-    }
-    __syncwarp();
+  if (tid < 64) {
+    const double* mk = w.kmean + (size_t)bh * kHeadDim;
+    double m = 0.0;
+    for (int c = 0; c < kHeadDim; ++c) m += (double)qt[c * kThreshPad + tid] * mk[c];
+    mu_s[tid] = (float)m;
+  }
+  const int ti = tid >> 4, tj = tid & 15;   // rows 4 ti .. 4 ti + 3, columns 8 tj .. 8 tj + 7
+  float y[4][8];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) y[a][c] = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < kHeadDim; ++d) {
+    const float4 qa = *reinterpret_cast<const float4*>(&qt[d * kThreshPad + 4 * ti]);
+    const float4 c0 = *reinterpret_cast<const float4*>(&cov_s[d * kHeadDim + 8 * tj]);
+    const float4 c1 = *reinterpret_cast<const float4*>(&cov_s[d * kHeadDim + 8 * tj + 4]);
+    const float av[4] = {qa.x, qa.y, qa.z, qa.w};
+    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) y[a][c] = fmaf(av[a], cv[c], y[a][c]);
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    float q = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) q = fmaf(qt[(8 * tj + c) * kThreshPad + 4 * ti + a], y[a][c], q);
+    part[4 * ti + a][tj] = q;
+  }
+  __syncthreads();
+  if (tid < 64 && i0 + tid < s.Nb) {
     double quad = 0.0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int c = lane + 32 * e;
-      double y = 0.0;
-      for (int d = 0; d < kHeadDim; ++d) y += (double)cov_s[d * kHeadDim + c] * qrow[warp][d];
-      quad += y * qrow[warp][c];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mu += __shfl_xor_sync(0xffffffffu, mu, o);
-      quad += __shfl_xor_sync(0xffffffffu, quad, o);
-    }
-    if (lane == 0) {
-      const double sd = (double)kScale;
-      const double m = sd * mu;
-      const double var = fmax(sd * sd * quad, 0.0);
-      w.thresh[(size_t)bh * s.Nb + i] = (float)(m + (double)tau * sqrt(var));
-    }
-    __syncwarp();
+    for (int c = 0; c < 16; ++c) quad += (double)part[tid][c];
+    const double sd = (double)kScale;
+    const double m = sd * (double)mu_s[tid];
+    const double var = fmax(sd * sd * quad, 0.0);
+    w.thresh[(size_t)bh * s.Nb + i0 + tid] = (float)(m + (double)tau * sqrt(var));
   }
 }
 
@@ -211,67 +259,69 @@ __global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau)
 // per-row counts reach memory).  Grid (ceil(Nb / 64), BH); a 64 x 64 tile of proxies per step,
 // 4 x 4 per thread from transposed shared-memory tiles.
 // -------------------------------------------------------------------------------------------------
-constexpr int kRoutePad = 68;
+constexpr int kRouteRows = 64, kRouteCols = 128;
+constexpr int kRoutePadQ = kRouteRows + 4, kRoutePadK = kRouteCols + 4;
 
-__global__ void __launch_bounds__(256) route_kernel(Shape s, Work w, int sink_b0, int sink_b1) {
-  extern __shared__ float rsm[];
-  float* Qt = rsm;                      // [128][68]
-  float* Kt = rsm + kHeadDim * kRoutePad;  // [128][68]
-  __shared__ float th[64];
-  __shared__ int cnt[64];
-  const int bh = blockIdx.y, i0 = blockIdx.x * 64, tid = threadIdx.x, lane = tid & 31;
-  const int ti = tid >> 4, tj = tid & 15;
+__global__ void __launch_bounds__(128) route_kernel(Shape s, Work w, int sink_b0, int sink_b1) {
+  extern __shared__ __align__(16) float rsm[];
+  float* Qt = rsm;                                  // [128][68]   Qbar^T of the 64 query blocks
+  float* Kt = rsm + kHeadDim * kRoutePadQ;          // [128][132]  Kbar^T of 128 key blocks
+  __shared__ float th[kRouteRows];
+  __shared__ int cnt[kRouteRows];
+  const int bh = blockIdx.y, i0 = blockIdx.x * kRouteRows, tid = threadIdx.x, lane = tid & 31;
+  const int ti = tid >> 4, tj = tid & 15;           // rows 8 ti .. 8 ti + 7, columns 8 tj .. 8 tj + 7
   const float* qb = w.qbar + (size_t)bh * s.Nb * kHeadDim;
   const float* kb = w.kbar + (size_t)bh * s.Nb * kHeadDim;
-  for (int idx = tid; idx < 64 * kHeadDim; idx += 256) {
+  for (int idx = tid; idx < kRouteRows * kHeadDim; idx += 128) {
     const int r = idx / kHeadDim, c = idx % kHeadDim;
-    Qt[c * kRoutePad + r] = (i0 + r < s.Nb) ? qb[(size_t)(i0 + r) * kHeadDim + c] : 0.f;
+    Qt[c * kRoutePadQ + r] = (i0 + r < s.Nb) ? qb[(size_t)(i0 + r) * kHeadDim + c] : 0.f;
   }
-  if (tid < 64) {
+  if (tid < kRouteRows) {
     th[tid] = (i0 + tid < s.Nb) ? w.thresh[(size_t)bh * s.Nb + i0 + tid] : 0.f;
     cnt[tid] = 0;
   }
-  for (int j0 = 0; j0 < s.Nb; j0 += 64) {
+  for (int j0 = 0; j0 < s.Nb; j0 += kRouteCols) {
     __syncthreads();
-    for (int idx = tid; idx < 64 * kHeadDim; idx += 256) {
+    for (int idx = tid; idx < kRouteCols * kHeadDim; idx += 128) {
       const int r = idx / kHeadDim, c = idx % kHeadDim;
-      Kt[c * kRoutePad + r] = (j0 + r < s.Nb) ? kb[(size_t)(j0 + r) * kHeadDim + c] : 0.f;
+      Kt[c * kRoutePadK + r] = (j0 + r < s.Nb) ? kb[(size_t)(j0 + r) * kHeadDim + c] : 0.f;
     }
     __syncthreads();
-    float acc[4][4];
+    float acc[8][8];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-#pragma unroll 4
+      for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+#pragma unroll 2
     for (int d = 0; d < kHeadDim; ++d) {
-      const float4 qa = *reinterpret_cast<const float4*>(&Qt[d * kRoutePad + 4 * ti]);
-      const float4 kk = *reinterpret_cast<const float4*>(&Kt[d * kRoutePad + 4 * tj]);
-      const float av[4] = {qa.x, qa.y, qa.z, qa.w};
-      const float bv[4] = {kk.x, kk.y, kk.z, kk.w};
+      const float4 q0 = *reinterpret_cast<const float4*>(&Qt[d * kRoutePadQ + 8 * ti]);
+      const float4 q1 = *reinterpret_cast<const float4*>(&Qt[d * kRoutePadQ + 8 * ti + 4]);
+      const float4 k0 = *reinterpret_cast<const float4*>(&Kt[d * kRoutePadK + 8 * tj]);
+      const float4 k1 = *reinterpret_cast<const float4*>(&Kt[d * kRoutePadK + 8 * tj + 4]);
+      const float av[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const float bv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(av[a], bv[c], acc[a][c]);
+        for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(av[a], bv[c], acc[a][c]);
     }
-    // 4 rows x 4 columns of decisions -> one nibble per row, OR-combined across the 8 lanes that
-    // share a 32-column word.
+    // 8 rows x 8 columns of decisions -> one byte per row, OR-combined across the 4 lanes that
+    // share a 32-column word (lanes differing in their two lowest bits).
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int il = 4 * ti + a;
+    for (int a = 0; a < 8; ++a) {
+      const int il = 8 * ti + a;
       const int i = i0 + il;
       uint32_t bits = 0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int jj = j0 + 4 * tj + c;
+      for (int c = 0; c < 8; ++c) {
+        const int jj = j0 + 8 * tj + c;
         const float shat = acc[a][c] * kScale;
-        if (jj < s.Nb && shat > th[il]) bits |= 1u << (4 * (tj & 7) + c);
+        if (jj < s.Nb && shat > th[il]) bits |= 1u << (8 * (tj & 3) + c);
       }
       bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
       bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
-      bits |= __shfl_xor_sync(0xffffffffu, bits, 4);
-      if ((lane & 7) == 0 && i < s.Nb) {
-        const int wd = (j0 >> 5) + (tj >> 3);
+      if ((lane & 3) == 0 && i < s.Nb) {
+        const int wd = (j0 >> 5) + (tj >> 2);
         if (wd < s.Nw) {
           const int jb = 32 * wd;
           for (int jj = max(i - 1, jb); jj <= min(i + 1, jb + 31); ++jj)
@@ -287,7 +337,7 @@ __global__ void __launch_bounds__(256) route_kernel(Shape s, Work w, int sink_b0
     }
   }
   __syncthreads();
-  if (tid < 64 && i0 + tid < s.Nb) {
+  if (tid < kRouteRows && i0 + tid < s.Nb) {
     const int c = cnt[tid];
     w.rowcount[(size_t)bh * s.Nb + i0 + tid] = c;
     atomicAdd(&w.stats[0], (unsigned long long)c);
@@ -309,31 +359,25 @@ __global__ void expand_mask_kernel(Shape s, Work w, unsigned char* out) {
 
 void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
                     const Work& w, bool anchors, cudaStream_t st) {
-  summary_kernel<<<dim3(s.Nb, s.B), 256, 0, st>>>(q, k, v, s, w, anchors ? 1 : 0);
+  summary_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, k, v, s, w, anchors ? 1 : 0);
 }
 
 void launch_kstats(const Shape& s, const Work& w, cudaStream_t st) {
-  kstats_kernel<<<dim3(kHeadDim / 16, s.BH), 256, 0, st>>>(s, w);
+  kmean_kernel<<<s.BH, kHeadDim, 0, st>>>(s, w);
+  kgram_kernel<<<dim3(kGramSplits, s.BH), 256, 0, st>>>(s, w, w.gram_partial);
+  kgram_reduce_kernel<<<dim3(kHeadDim * kHeadDim / 256, s.BH), 256, 0, st>>>(s, w, w.gram_partial);
 }
 
 void launch_thresh(const Shape& s, const Work& w, float tau, cudaStream_t st) {
-  const int smem = kHeadDim * kHeadDim * sizeof(float);
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(thresh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    configured = true;
-  }
+  const int smem = (kHeadDim * kHeadDim + kHeadDim * kThreshPad) * sizeof(float);
+  cudaFuncSetAttribute(thresh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   thresh_kernel<<<dim3((s.Nb + 63) / 64, s.BH), 256, smem, st>>>(s, w, tau);
 }
 
 void launch_route(const Shape& s, const Work& w, int sink_b0, int sink_b1, cudaStream_t st) {
-  const int smem = 2 * kHeadDim * kRoutePad * sizeof(float);
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    configured = true;
-  }
-  route_kernel<<<dim3((s.Nb + 63) / 64, s.BH), 256, smem, st>>>(s, w, sink_b0, sink_b1);
+  const int smem = kHeadDim * (kRoutePadQ + kRoutePadK) * sizeof(float);
+  cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  route_kernel<<<dim3((s.Nb + kRouteRows - 1) / kRouteRows, s.BH), 128, smem, st>>>(s, w, sink_b0, sink_b1);
 }
 
 void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, cudaStream_t st) {

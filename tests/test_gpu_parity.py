@@ -150,4 +150,4 @@ def test_stream_and_stats_and_timing():
     assert ms > 0
     exact, total, mn, mx = sa.last_stats()
     assert total == 2 * 32 * 32 and 0 < exact <= total and 2 <= mn <= mx <= 32
-    assert sa.last_launch_count() == 5
+    assert sa.last_launch_count() == 7
