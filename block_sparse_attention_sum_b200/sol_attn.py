@@ -29,6 +29,7 @@ EXPORTS = [
     "sol_attn_kernel_ms_sum",
     "sol_attn_last_launch_count",
     "sol_attn_release_workspace",
+    "sol_attn_fwd_noalloc",
 ]
 
 STATUS = {
@@ -81,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_last_launch_count.restype = i
     lib.sol_attn_release_workspace.argtypes = []
     lib.sol_attn_release_workspace.restype = None
+    lib.sol_attn_fwd_noalloc.argtypes = fwd_args
+    lib.sol_attn_fwd_noalloc.restype = i
     _lib = lib
     return lib
 
@@ -131,6 +134,13 @@ def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, strea
 def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
     """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
     return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream)
+
+
+def sol_attn_fwd_noalloc(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
+    """Allocation-free Sol-Attn forward (library-owned fixed scratch; see include/sol_attn.h).
+
+    ``out`` should be preallocated by a caller that cannot allocate during the call."""
+    return _fwd("sol_attn_fwd_noalloc", q, k, v, tau, sink_start, sink_tokens, out, stream)
 
 
 def sol_attn(q, k, v, tau=1.0, sink_start=None, sink_tokens=0, out=None):

@@ -126,6 +126,27 @@ int sol_attn_last_launch_count(void);
 /* Frees this process's workspaces on every device (synchronises each device first). */
 void sol_attn_release_workspace(void);
 
+/*
+ * Allocation-free variant of sol_attn_fwd (the pages have no counterpart: this serves callers that
+ * cannot allocate device memory during the call, e.g. code running inside a memory pool that
+ * forbids outside allocations or a runtime that reserved all device memory up front).
+ *   - Same arguments, layout, results and argument errors as sol_attn_fwd.
+ *   - Its scratch is a fixed 64 MiB region declared at file scope in the library (plus two small
+ *     status / statistics words); every GPU that loads the library holds it until the process
+ *     exits.  The call never calls cudaMalloc / cudaFree or any allocating routine.  A shape whose
+ *     scratch exceeds 64 MiB (for example B*H = 32 at N > ~40K tokens) returns SOL_ERR_SHAPE with a
+ *     message; use sol_attn_fwd for those.
+ *   - The first call on a device (with that device current) looks up the scratch region's device
+ *     address; make that first call before any stream capture on the device.
+ *   - All calls share the one region: calls that overlap on the GPU (different streams, or several
+ *     host threads) race and must be serialised by the caller.  The region keeps the last call's
+ *     contents; everything a call needs zeroed it clears itself.
+ *   - Not covered by sol_attn_last_stats / sol_attn_get_device_status / kernel timing (those
+ *     report the pooled-workspace entry points).
+ */
+int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                         int sink_start, int sink_tokens, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
