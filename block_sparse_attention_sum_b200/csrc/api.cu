@@ -343,6 +343,7 @@ int sol_attn_get_device_status(void* stream) {
       cudaMemset(d->status, 0, sizeof(int)) != cudaSuccess)
     return fail(SOL_ERR_LAUNCH, "status read failed");
   if (h == kDevTimeout) return fail(SOL_ERR_TIMEOUT, "a bounded wait inside a kernel ran out");
+  if (h == kDevMisaligned) return fail(SOL_ERR_LAUNCH, "shared memory window misaligned; the kernel did not run");
   return SOL_OK;
 }
 

@@ -17,11 +17,13 @@
 //    for the columns that are exact for the row's block.  n_j exp(a_j) and exp(a_j) n_j Vbar_j =
 //    exp(a_j) Vhat_j are exactly the surrogate's denominator and numerator terms.
 //  * Warp roles: warp 0 TMA producer (derives the tile list from the routing bitmask), warp 1 TMEM
-//    owner and MMA issuer, warps 4-7 softmax / O-correction / epilogue (one thread per query row,
-//    TMEM lane = row).  S is double-buffered in TMEM; O accumulates in TMEM.
+//    owner and S = Q K^T issuer, warp 2 O += P V issuer, warps 4-11 two softmax warpgroups (TMEM
+//    lane = row; each warpgroup owns 64 of the 128 columns of S, P and O).  S and P are
+//    double-buffered in TMEM; O accumulates in TMEM.
 //  * Online softmax in base 2 with a lazily updated reference max: O and l are rescaled only when a
 //    row's max grows by more than 2^8, which keeps every probability <= 256.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cfloat>
 
 #include "attn_fwd.cuh"
@@ -54,19 +56,69 @@ struct __align__(1024) FwdSmem {
   TileDesc desc[kDescRing];
   uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
   uint64_t dfull[kDescRing];
-  uint64_t qfull, sfull[2], sfree[2], pready, pvdone, mmadone;
-  float lsum[2][128];
+  uint64_t qfull, sfull[2], sfree[2], pready, pvdone, mmadone, mmadone2;
+  uint64_t xbar[2], lbar;   // softmax warpgroups: row-max exchange per S parity, row-sum exchange
+  float xmax[2][2][128];   // [S buffer][warpgroup][row] partial row maxima; row sums at the end
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr size_t kSmemBytes = sizeof(FwdSmem) + 1024;
+// The dynamic shared-memory window starts 1024-byte aligned on sm_100 (checked at run time: a
+// misaligned base is reported through the status word and the CTA exits without touching memory).
+constexpr size_t kSmemBytes = sizeof(FwdSmem);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed FP32 pairs (sm_100 f32x2 arithmetic).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 unf2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^y for a pair on the FMA pipe, to take load off the MUFU unit (16 results / clk / SM).
+// Range reduction y = n + f with n = round(y) (via the 1.5 * 2^23 rounding constant), f in
+// [-1/2, 1/2]; 2^f by a cubic fitted to minimise the relative error on [-1/2, 1/2] (Lawson's
+// iteration, max relative error 1.0e-4, below BF16's 2^-9); 2^n by adding n to the exponent field.
+// Inputs below -127 (and -inf) are clamped, giving 0.
+__device__ __forceinline__ float2 exp2_poly_pair(float y0, float y1) {
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  const uint64_t yy = f2(fmaxf(y0, -127.f), fmaxf(y1, -127.f));
+  const uint64_t t = add2(yy, f2(kRound, kRound));
+  const uint64_t n = add2(t, f2(-kRound, -kRound));
+  const uint64_t fr = fma2(n, f2(-1.f, -1.f), yy);
+  uint64_t p = fma2(f2(0.05500893294811249f, 0.05500893294811249f), fr, f2(0.2422109693288803f, 0.2422109693288803f));
+  p = fma2(p, fr, f2(0.6932829022407532f, 0.6932829022407532f));
+  p = fma2(p, fr, f2(1.f, 1.f));
+  const float2 pf = unf2(p), tf = unf2(t);
+  return make_float2(__int_as_float(__float_as_int(pf.x) + (__float_as_int(tf.x) << 23)),
+                     __int_as_float(__float_as_int(pf.y) + (__float_as_int(tf.y) << 23)));
 }
 
 __device__ __forceinline__ void set_timeout(int* status) { atomicExch(status, kDevTimeout); }
@@ -78,9 +130,13 @@ __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
                     const __grid_constant__ CUtensorMap tm_vp, const FwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  FwdSmem& sm = *reinterpret_cast<FwdSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(smem_raw) & 1023u) {   // uniform across the CTA
+    if (tid == 0) atomicExch(p.status, kDevMisaligned);
+    return;
+  }
+  FwdSmem& sm = *reinterpret_cast<FwdSmem*>(smem_raw);
   volatile int* abort = &sm.abort;
 
   const int unit = p.order ? p.order[blockIdx.x] : (int)blockIdx.x;
@@ -105,6 +161,10 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&sm.pready, 256);
     mbar_init(&sm.pvdone, 1);
     mbar_init(&sm.mmadone, 1);
+    mbar_init(&sm.mmadone2, 1);
+    mbar_init(&sm.xbar[0], 256);
+    mbar_init(&sm.xbar[1], 256);
+    mbar_init(&sm.lbar, 256);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -232,27 +292,10 @@ __global__ void __launch_bounds__(384, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------------------- MMA issuer
+    // --------------------------------------------------------------------------- S = Q K^T issuer
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qfull, 0, abort);
       const uint32_t q_base = smem_u32(&sm.q[0][0]);
-      uint32_t prev_kind = kTilePair;
-      auto issue_pv = [&](int u, uint32_t kind) {
-        const int s = u % kStages;
-        if (!mbar_wait(&sm.pready, u & 1, abort) || !mbar_wait(&sm.vfull[s], (u / kStages) & 1, abort)) return false;
-        tc_fence_after();
-        const int nsteps = kind == kTileSingle ? 4 : 8;
-        const uint32_t idesc = idesc_bf16(128, 128, false, true);
-        const uint32_t v_base = smem_u32(&sm.v[s][0][0]);
-        const uint32_t p_col = tmem + kColP + 64 * (u & 1);
-        for (int kk = 0; kk < nsteps; ++kk) {
-          const uint64_t bd = sdesc_sw128(v_base + kk * 2048, kTileBytes, 1024);
-          umma_ts(tmem + kColO, p_col + 8 * kk, bd, idesc, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&sm.vempty[s]);
-        umma_commit(&sm.pvdone);
-        return true;
-      };
       for (int t = 0; ok; ++t) {
         const int s = t % kStages;
         if (!mbar_wait(&sm.kfull[s], (t / kStages) & 1, abort)) {
@@ -276,19 +319,43 @@ __global__ void __launch_bounds__(384, 1)
         }
         umma_commit(&sm.sfull[bsel]);
         umma_commit(&sm.kempty[s]);
-        if (t > 0 && !issue_pv(t - 1, prev_kind)) {
-          ok = false;
-          break;
-        }
-        prev_kind = d.kind;
-        if (d.flags & 0x100u) {
-          ok = issue_pv(t, d.kind);
-          break;
-        }
+        if (d.flags & 0x100u) break;
       }
       if (!ok) set_timeout(p.status);
       umma_commit(&sm.mmadone);
       mbar_wait(&sm.mmadone, 0, abort);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------------------ O += P V issuer
+    // A separate issuing thread, so that P V of a tile goes to the tensor core as soon as its P is
+    // ready instead of queueing behind the next Q K^T in one thread's program order.
+    if (lane == 0) {
+      bool ok = true;
+      for (int u = 0; ok; ++u) {
+        const int s = u % kStages;
+        if (!mbar_wait(&sm.dfull[u % kDescRing], (u / kDescRing) & 1, abort) || !mbar_wait(&sm.pready, u & 1, abort) ||
+            !mbar_wait(&sm.vfull[s], (u / kStages) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        const TileDesc d = sm.desc[u % kDescRing];
+        tc_fence_after();
+        const int nsteps = d.kind == kTileSingle ? 4 : 8;
+        const uint32_t idesc = idesc_bf16(128, 128, false, true);
+        const uint32_t v_base = smem_u32(&sm.v[s][0][0]);
+        const uint32_t p_col = tmem + kColP + 64 * (u & 1);
+        for (int kk = 0; kk < nsteps; ++kk) {
+          const uint64_t bd = sdesc_sw128(v_base + kk * 2048, kTileBytes, 1024);
+          umma_ts(tmem + kColO, p_col + 8 * kk, bd, idesc, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&sm.vempty[s]);
+        umma_commit(&sm.pvdone);
+        if (d.flags & 0x100u) break;
+      }
+      if (!ok) set_timeout(p.status);
+      umma_commit(&sm.mmadone2);
+      mbar_wait(&sm.mmadone2, 0, abort);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -320,107 +387,90 @@ __global__ void __launch_bounds__(384, 1)
       const TileDesc d = sm.desc[t % kDescRing];
       tc_fence_after();
       const bool single = d.kind == kTileSingle;
-      uint32_t own[64], oth[32];
+      uint32_t own[64];
       const uint32_t s_addr = lane_addr + kColS + 128 * bsel;
-      const uint32_t oth_addr = s_addr + 64 * (1 - wg);
-      const bool have_own = !single || wg == 0, have_oth = !single || wg == 1;
-      if (have_own) {
+      const bool pooled = d.kind == kTilePooled;
+      // columns of this thread's half that are valid for its row (warp-uniform)
+      int lim_own = 64;
+      if (!pooled) {
+        const bool v0 = (d.flags >> hf) & 1u;
+        const bool v1 = !single && ((d.flags >> (2 + hf)) & 1u);
+        const int lim0 = v0 ? min(64, p.N - 64 * d.j0) : 0;
+        const int lim1 = v1 ? min(64, p.N - 64 * d.j1) : 0;
+        lim_own = wg ? lim1 : lim0;
+      }
+      if (lim_own > 0) {
         tmem_ld32_at<0>(s_addr + 64 * wg, own);
         tmem_ld32_at<32>(s_addr + 64 * wg + 32, own);
+        tmem_ld_wait();
       }
-
-      // x: own columns (in place over the raw scores); the other half only feeds the row max.
-      // Exact tiles keep raw scores (the scale is folded into the exponent), pooled tiles carry
-      // scale and log2(n_j) bias.
+      tc_fence_before();
+      mbar_arrive(&sm.sfree[bsel]);
+      // x: this thread's 64 columns in place over the raw scores.  Exact tiles keep raw scores (the
+      // base-2 scale is folded into the exponent), pooled tiles carry scale and the log2(n_j) bias.
       float* x = reinterpret_cast<float*>(own);
       float mp[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mp[k] = -INFINITY;
-      if (d.kind == kTilePooled) {
-        uint32_t mw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int wd = 4 * d.j0 + e;
-          mw[e] = wd < p.Nw ? mrow[wd] : 0xffffffffu;
-        }
-        const int jb_own = 128 * d.j0 + 64 * wg, jb_oth = 128 * d.j0 + 64 * (1 - wg);
-        const uint32_t m_own0 = wg ? mw[2] : mw[0], m_own1 = wg ? mw[3] : mw[1];
-        const uint32_t m_oth0 = wg ? mw[0] : mw[2], m_oth1 = wg ? mw[1] : mw[3];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tmem_ld32_at<0>(oth_addr + 32 * half, oth);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int jo = jb_oth + 32 * half + c;
-            const float bo = (jo == p.Nb - 1) ? lg_last : 6.0f;
-            const bool ex = ((half ? m_oth1 : m_oth0) >> c) & 1u;
-            const float yv = (jo < p.Nb && !ex) ? fmaf(__uint_as_float(oth[c]), sc, bo) : -INFINITY;
-            mp[c & 7] = fmaxf(mp[c & 7], yv);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&sm.sfree[bsel]);
+      if (pooled) {
+        const int jb_own = 128 * d.j0 + 64 * wg;
+        const int wd0 = 4 * d.j0 + 2 * wg;
+        const uint32_t m_own0 = wd0 < p.Nw ? mrow[wd0] : 0xffffffffu;
+        const uint32_t m_own1 = wd0 + 1 < p.Nw ? mrow[wd0 + 1] : 0xffffffffu;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int j = jb_own + c;
           const float bias = (j == p.Nb - 1) ? lg_last : 6.0f;
           const bool ex = (((c < 32) ? m_own0 : m_own1) >> (c & 31)) & 1u;
-          x[c] = (j < p.Nb && !ex) ? fmaf(__uint_as_float(own[c]), sc, bias) : -INFINITY;
-          mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+          x[c] = (j < p.Nb && !ex) ? fmaf(x[c], sc, bias) : -INFINITY;
         }
-      } else {
-        // block of each half and whether it is exact for this row's query block
-        const bool v0 = (d.flags >> hf) & 1u;
-        const bool v1 = !single && ((d.flags >> (2 + hf)) & 1u);
-        const int lim0 = v0 ? p.N - 64 * d.j0 : 0;
-        const int lim1 = v1 ? p.N - 64 * d.j1 : 0;
-        const int lim_own = wg ? lim1 : lim0, lim_oth = wg ? lim0 : lim1;
-        if (have_oth) {
+      } else if (lim_own < 64) {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            tmem_ld32_at<0>(oth_addr + 32 * half, oth);
-            tmem_ld_wait();
-            const int lim = lim_oth - 32 * half;
-            if (lim >= 32) {
+        for (int c = 0; c < 64; ++c) x[c] = c < lim_own ? x[c] : -INFINITY;
+      }
+      if (lim_own > 0) {
 #pragma unroll
-              for (int c = 0; c < 32; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(oth[c]));
-            } else if (lim > 0) {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) mp[c & 7] = fmaxf(mp[c & 7], c < lim ? __uint_as_float(oth[c]) : -INFINITY);
-            }
-          }
-        } else {
-          tmem_ld_wait();
-        }
-        tc_fence_before();
-        mbar_arrive(&sm.sfree[bsel]);
-        if (lim_own < 64) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = c < lim_own ? x[c] : -INFINITY;
-        }
-#pragma unroll
-        for (int c = 0; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+        for (int c = 0; c < 64; c += 2) mp[(c >> 1) & 7] = max3(mp[(c >> 1) & 7], x[c], x[c + 1]);
       }
       float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      const bool pooled = d.kind == kTilePooled;
       if (!pooled) mx *= sc;   // exact tiles: raw scores, base-2 scale applied here
+      // the row max over both halves: exchange with the other warpgroup's thread of this row
+      sm.xmax[bsel][wg][r] = mx;
+      mbar_arrive(&sm.xbar[bsel]);
+      if (!mbar_wait(&sm.xbar[bsel], (t >> 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      mx = fmaxf(mx, sm.xmax[bsel][1 - wg][r]);
       const float m_new = fmaxf(m_ref, mx);
       const bool upd = m_new > m_ref + 8.0f;
       const float m_use = upd ? m_new : m_ref;
       const float m_sub = m_use == -INFINITY ? 0.f : m_use;
       const float alpha = upd ? ex2(m_ref - m_sub) : 1.f;
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t rs2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
       uint32_t pk[32];
-      const float fs = pooled ? 1.f : sc;
+      if (lim_own > 0) {
+        const float fs = pooled ? 1.f : sc;
+        const uint64_t fs2 = f2(fs, fs), nm2 = f2(-m_sub, -m_sub);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2(fmaf(x[2 * c], fs, -m_sub));
-        const float p1 = ex2(fmaf(x[2 * c + 1], fs, -m_sub));
-        rs[c & 3] += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < 32; ++c) {
+          const float2 y = unf2(fma2(f2(x[2 * c], x[2 * c + 1]), fs2, nm2));
+          float2 pp;
+          if ((c & 3) == 3) {
+            pp = exp2_poly_pair(y.x, y.y);
+          } else {
+            pp.x = ex2(y.x);
+            pp.y = ex2(y.y);
+          }
+          rs2[c & 1] = add2(rs2[c & 1], f2(pp.x, pp.y));
+          pk[c] = pack_bf16x2(pp.x, pp.y);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      const float2 rsa = unf2(add2(rs2[0], rs2[1]));
+      l = l * alpha + (rsa.x + rsa.y);
       // P buffer (t & 1) was last read by P V of tile t - 2; O must be quiet before rescaling
       if (t > 0 && !mbar_wait(&sm.pvdone, (t - 1) & 1, abort)) {
         ok = false;
@@ -451,10 +501,17 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && !mbar_wait(&sm.pvdone, t & 1, abort)) ok = false;
     if (!ok) set_timeout(p.status);
     tc_fence_after();
-    // combine the two halves' row sums
-    sm.lsum[wg][r] = l;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    l = sm.lsum[0][r] + sm.lsum[1][r];
+    // combine the two halves' row sums (the max-exchange buffer of the other S parity is free: both
+    // warpgroups read it, for tile t - 1, before arriving at the exchange of tile t)
+    if (ok) {
+      sm.xmax[(t + 1) & 1][wg][r] = l;
+      mbar_arrive(&sm.lbar);
+      if (mbar_wait(&sm.lbar, 0, abort))
+        l = sm.xmax[(t + 1) & 1][0][r] + sm.xmax[(t + 1) & 1][1][r];
+      else
+        ok = false;
+    }
+    if (!ok) set_timeout(p.status);
     if (__all_sync(0xffffffffu, ok)) {
       // epilogue: o = O / l (Sol-Attn2: merged with the anchor's complementary tail)
       float scale_o = 1.f / l;

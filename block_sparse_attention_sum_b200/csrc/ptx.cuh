@@ -12,6 +12,7 @@ namespace sol {
 enum : int {
   kDevOk = 0,
   kDevTimeout = 1,
+  kDevMisaligned = 2,   // dynamic shared memory not 1024-byte aligned
 };
 
 // Upper bound on any single mbarrier wait, in nanoseconds of %globaltimer (about one second).
