@@ -38,8 +38,9 @@ constexpr int kDescRing = 8;                   // tile descriptors in flight (pr
                                                // the MMAs, MMAs <= 2 ahead of the softmax)
 constexpr uint32_t kTileBytes = 128 * 64 * 2;  // 128 rows x 64 BF16 columns (one swizzled half, 16 KB)
 constexpr uint32_t kBoxBytes = 64 * 64 * 2;    // one 64-row x 64-column BF16 TMA box (8 KB)
-// TMEM columns: S double buffer, O accumulator, P double buffer (BF16 pairs)
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+// TMEM columns: S double buffer (P of each half is written over that half's S columns once they
+// are read), and one O accumulator per softmax warpgroup (each over its half of every tile's keys).
+constexpr uint32_t kColS = 0, kColO = 256;
 
 enum : uint32_t { kTilePair = 0, kTileSingle = 1, kTilePooled = 2 };
 
@@ -56,9 +57,9 @@ struct __align__(1024) FwdSmem {
   TileDesc desc[kDescRing];
   uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
   uint64_t dfull[kDescRing];
-  uint64_t qfull, sfull[2], sfree[2], pready, pvdone, mmadone, mmadone2;
-  uint64_t xbar[2], lbar;   // softmax warpgroups: row-max exchange per S parity, row-sum exchange
-  float xmax[2][2][128];   // [S buffer][warpgroup][row] partial row maxima; row sums at the end
+  uint64_t qfull, sfull[2], sfree[2], pready[2], pvdone[2], mmadone, mmadone2;
+  uint64_t lbar;            // softmax warpgroups: (max, sum) exchange before the epilogue merge
+  float xm[2][128], xl[2][128];   // [warpgroup][row] running max and row sum, for the epilogue merge
   uint32_t tmem_base;
   int abort;
 };
@@ -156,14 +157,12 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&sm.qfull, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.sfull[i], 1);
-      mbar_init(&sm.sfree[i], 256);
+      mbar_init(&sm.sfree[i], 1);
+      mbar_init(&sm.pready[i], 128);
+      mbar_init(&sm.pvdone[i], 1);
     }
-    mbar_init(&sm.pready, 256);
-    mbar_init(&sm.pvdone, 1);
     mbar_init(&sm.mmadone, 1);
     mbar_init(&sm.mmadone2, 1);
-    mbar_init(&sm.xbar[0], 256);
-    mbar_init(&sm.xbar[1], 256);
     mbar_init(&sm.lbar, 256);
     sm.abort = 0;
     fence_mbar_init();
@@ -219,20 +218,6 @@ __global__ void __launch_bounds__(384, 1)
               tma_load_4d(&sm.k[s][dh][slot * 64 * 64], &tm_k, &sm.kfull[s], 64 * dh, h, 64 * (slot ? d.j1 : d.j0),
                           b);
         }
-        if (t >= kStages && !mbar_wait(&sm.vempty[s], ph, abort)) {
-          ok = false;
-          ++t;   // the K copy of this tile is in flight
-          return;
-        }
-        mbar_arrive_expect_tx(&sm.vfull[s], bytes);
-        if (pooled) {
-          for (int dh = 0; dh < 2; ++dh) tma_load_3d(&sm.v[s][dh][0], &tm_vp, &sm.vfull[s], 64 * dh, 128 * d.j0, bh);
-        } else {
-          for (int slot = 0; slot < nblk; ++slot)
-            for (int dh = 0; dh < 2; ++dh)
-              tma_load_4d(&sm.v[s][dh][slot * 64 * 64], &tm_v, &sm.vfull[s], 64 * dh, h, 64 * (slot ? d.j1 : d.j0),
-                          b);
-        }
         ++t;
       };
       auto push = [&](TileDesc d) {
@@ -284,10 +269,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok) set_timeout(p.status);
       // never leave the CTA with bulk copies in flight
-      for (int u = max(0, t - kStages); u < t; ++u) {
-        mbar_wait(&sm.kfull[u % kStages], (u / kStages) & 1, abort);
-        mbar_wait(&sm.vfull[u % kStages], (u / kStages) & 1, abort);
-      }
+      for (int u = max(0, t - kStages); u < t; ++u) mbar_wait(&sm.kfull[u % kStages], (u / kStages) & 1, abort);
       mbar_wait(&sm.qfull, 0, abort);
     }
     __syncwarp();
@@ -304,6 +286,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         const TileDesc d = sm.desc[t % kDescRing];
         const int bsel = t & 1;
+        // the buffer's previous tile (t - 2): its P was read by that tile's P V
         if (t >= 2 && !mbar_wait(&sm.sfree[bsel], ((t >> 1) - 1) & 1, abort)) {
           ok = false;
           break;
@@ -328,29 +311,44 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------------------------ O += P V issuer
-    // A separate issuing thread, so that P V of a tile goes to the tensor core as soon as its P is
-    // ready instead of queueing behind the next Q K^T in one thread's program order.
+    // One product per softmax warpgroup and tile: O_w += P_w V_w over the warpgroup's 64 keys, issued
+    // as soon as that warpgroup's P is in TMEM.  A separate thread from the Q K^T issuer, so neither
+    // queues behind the other in program order.
     if (lane == 0) {
       bool ok = true;
+      bool b_started = false;
       for (int u = 0; ok; ++u) {
         const int s = u % kStages;
-        if (!mbar_wait(&sm.dfull[u % kDescRing], (u / kDescRing) & 1, abort) || !mbar_wait(&sm.pready, u & 1, abort) ||
+        const int bsel = u & 1;
+        if (!mbar_wait(&sm.dfull[u % kDescRing], (u / kDescRing) & 1, abort) ||
             !mbar_wait(&sm.vfull[s], (u / kStages) & 1, abort)) {
           ok = false;
           break;
         }
         const TileDesc d = sm.desc[u % kDescRing];
-        tc_fence_after();
-        const int nsteps = d.kind == kTileSingle ? 4 : 8;
         const uint32_t idesc = idesc_bf16(128, 128, false, true);
         const uint32_t v_base = smem_u32(&sm.v[s][0][0]);
-        const uint32_t p_col = tmem + kColP + 64 * (u & 1);
-        for (int kk = 0; kk < nsteps; ++kk) {
-          const uint64_t bd = sdesc_sw128(v_base + kk * 2048, kTileBytes, 1024);
-          umma_ts(tmem + kColO, p_col + 8 * kk, bd, idesc, (u > 0 || kk > 0) ? 1u : 0u);
+        for (int w = 0; w < 2 && ok; ++w) {
+          if (!mbar_wait(&sm.pready[w], u & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const bool skip = (w == 1 && d.kind == kTileSingle);   // no keys in the second half
+          if (!skip) {
+            const uint32_t p_col = tmem + kColS + 128 * bsel + 64 * w;   // P_w over its S columns
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = sdesc_sw128(v_base + (4 * w + kk) * 2048, kTileBytes, 1024);
+              const bool acc = w == 0 ? (u > 0 || kk > 0) : (b_started || kk > 0);
+              umma_ts(tmem + kColO + 128 * w, p_col + 8 * kk, bd, idesc, acc ? 1u : 0u);
+            }
+            if (w == 1) b_started = true;
+          }
+          umma_commit(&sm.pvdone[w]);
         }
+        if (!ok) break;
+        umma_commit(&sm.sfree[bsel]);
         umma_commit(&sm.vempty[s]);
-        umma_commit(&sm.pvdone);
         if (d.flags & 0x100u) break;
       }
       if (!ok) set_timeout(p.status);
@@ -358,11 +356,48 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(&sm.mmadone2, 0, abort);
     }
     __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------------------------------------------ V producer
+    // Loads V tiles in the order the K producer published them, so that K tiles (needed first, by
+    // Q K^T) never wait behind the release of a V stage.
+    if (lane == 0) {
+      bool ok = true;
+      int u = 0;
+      for (;; ++u) {
+        const int s = u % kStages;
+        if (!mbar_wait(&sm.dfull[u % kDescRing], (u / kDescRing) & 1, abort) ||
+            (u >= kStages && !mbar_wait(&sm.vempty[s], ((u / kStages) - 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
+        const TileDesc d = sm.desc[u % kDescRing];
+        const bool pooled = d.kind == kTilePooled;
+        const int nblk = d.kind == kTilePair ? 2 : 1;
+        mbar_arrive_expect_tx(&sm.vfull[s], pooled ? 2 * kTileBytes : 2 * kBoxBytes * nblk);
+        if (pooled) {
+          for (int dh = 0; dh < 2; ++dh) tma_load_3d(&sm.v[s][dh][0], &tm_vp, &sm.vfull[s], 64 * dh, 128 * d.j0, bh);
+        } else {
+          for (int slot = 0; slot < nblk; ++slot)
+            for (int dh = 0; dh < 2; ++dh)
+              tma_load_4d(&sm.v[s][dh][slot * 64 * 64], &tm_v, &sm.vfull[s], 64 * dh, h, 64 * (slot ? d.j1 : d.j0),
+                          b);
+        }
+        if (d.flags & 0x100u) {
+          ++u;
+          break;
+        }
+      }
+      if (!ok) set_timeout(p.status);
+      // never leave the CTA with bulk copies in flight
+      for (int w = max(0, u - kStages); w < u; ++w) mbar_wait(&sm.vfull[w % kStages], (w / kStages) & 1, abort);
+    }
+    __syncwarp();
   } else if (warp >= 4) {
     // --------------------------------------------------------------- softmax / correction / epilogue
     // Two warpgroups share the 128 rows (TMEM lane = row); warpgroup wg owns columns 64 wg .. 64 wg + 63
-    // of S, P and O.  Both compute the full row max (so they agree on the reference max without
-    // exchanging it) and exponentiate only their own half; their partial row sums are added at the end.
+    // of every tile and keeps its own online-softmax state (m, l) and its own O accumulator over
+    // those keys.  The two partial results of a row are merged exactly in the epilogue, so the
+    // warpgroups never wait for each other inside the tile loop.
     const int wg = (warp - 4) >> 2;
     const int r = ((warp & 3) << 5) | lane;   // query row within the tile == TMEM lane
     const int hf = r >> 6;
@@ -370,12 +405,14 @@ __global__ void __launch_bounds__(384, 1)
     const int tok = 64 * qb0 + r;
     const bool row_valid = tok < p.N;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t o_addr = lane_addr + kColO + 128 * wg;
     const uint32_t* mrow = p.mask + ((size_t)bh * p.Nb + min(qi, p.Nb - 1)) * p.Nw;
     const float sc = kScale * kLog2e;
     const int n_last = p.N - 64 * (p.Nb - 1);
     const float lg_last = log2f((float)n_last);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    bool o1_written = false;   // O_1 receives a product for every tile with a second 64-key half
     int t = 0;
     for (;; ++t) {
       const int bsel = t & 1;
@@ -387,61 +424,51 @@ __global__ void __launch_bounds__(384, 1)
       const TileDesc d = sm.desc[t % kDescRing];
       tc_fence_after();
       const bool single = d.kind == kTileSingle;
-      uint32_t own[64];
-      const uint32_t s_addr = lane_addr + kColS + 128 * bsel;
+      o1_written = o1_written || !single;
       const bool pooled = d.kind == kTilePooled;
-      // columns of this thread's half that are valid for its row (warp-uniform)
+      const uint32_t s_addr = lane_addr + kColS + 128 * bsel + 64 * wg;
+      // columns of this warpgroup's half that are valid for its row (warp-uniform)
       int lim_own = 64;
       if (!pooled) {
-        const bool v0 = (d.flags >> hf) & 1u;
-        const bool v1 = !single && ((d.flags >> (2 + hf)) & 1u);
-        const int lim0 = v0 ? min(64, p.N - 64 * d.j0) : 0;
-        const int lim1 = v1 ? min(64, p.N - 64 * d.j1) : 0;
-        lim_own = wg ? lim1 : lim0;
+        const bool v = wg ? (!single && ((d.flags >> (2 + hf)) & 1u)) : ((d.flags >> hf) & 1u);
+        const int jo = wg ? d.j1 : d.j0;
+        lim_own = v ? min(64, p.N - 64 * jo) : 0;
       }
+      uint32_t own[64];
       if (lim_own > 0) {
-        tmem_ld32_at<0>(s_addr + 64 * wg, own);
-        tmem_ld32_at<32>(s_addr + 64 * wg + 32, own);
+        tmem_ld32_at<0>(s_addr, own);
+        tmem_ld32_at<32>(s_addr + 32, own);
         tmem_ld_wait();
       }
-      tc_fence_before();
-      mbar_arrive(&sm.sfree[bsel]);
-      // x: this thread's 64 columns in place over the raw scores.  Exact tiles keep raw scores (the
-      // base-2 scale is folded into the exponent), pooled tiles carry scale and the log2(n_j) bias.
+      // x: this warpgroup's 64 columns in place over the raw scores.  Exact tiles keep raw scores
+      // (the base-2 scale is folded into the exponent), pooled tiles carry scale and log2(n_j) bias.
       float* x = reinterpret_cast<float*>(own);
-      float mp[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mp[k] = -INFINITY;
-      if (pooled) {
-        const int jb_own = 128 * d.j0 + 64 * wg;
-        const int wd0 = 4 * d.j0 + 2 * wg;
-        const uint32_t m_own0 = wd0 < p.Nw ? mrow[wd0] : 0xffffffffu;
-        const uint32_t m_own1 = wd0 + 1 < p.Nw ? mrow[wd0 + 1] : 0xffffffffu;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int j = jb_own + c;
-          const float bias = (j == p.Nb - 1) ? lg_last : 6.0f;
-          const bool ex = (((c < 32) ? m_own0 : m_own1) >> (c & 31)) & 1u;
-          x[c] = (j < p.Nb && !ex) ? fmaf(x[c], sc, bias) : -INFINITY;
-        }
-      } else if (lim_own < 64) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = c < lim_own ? x[c] : -INFINITY;
-      }
+      float mx = -INFINITY;
       if (lim_own > 0) {
+        if (pooled) {
+          const int jb_own = 128 * d.j0 + 64 * wg;
+          const int wd0 = 4 * d.j0 + 2 * wg;
+          const uint32_t m_own0 = wd0 < p.Nw ? mrow[wd0] : 0xffffffffu;
+          const uint32_t m_own1 = wd0 + 1 < p.Nw ? mrow[wd0 + 1] : 0xffffffffu;
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) mp[(c >> 1) & 7] = max3(mp[(c >> 1) & 7], x[c], x[c + 1]);
+          for (int c = 0; c < 64; ++c) {
+            const int j = jb_own + c;
+            const float bias = (j == p.Nb - 1) ? lg_last : 6.0f;
+            const bool ex = (((c < 32) ? m_own0 : m_own1) >> (c & 31)) & 1u;
+            x[c] = (j < p.Nb && !ex) ? fmaf(x[c], sc, bias) : -INFINITY;
+          }
+        } else if (lim_own < 64) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) x[c] = c < lim_own ? x[c] : -INFINITY;
+        }
+        float mp[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = x[k];
+#pragma unroll
+        for (int c = 8; c < 64; c += 2) mp[(c >> 1) & 7] = max3(mp[(c >> 1) & 7], x[c], x[c + 1]);
+        mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        if (!pooled) mx *= sc;   // exact tiles: raw scores, base-2 scale applied here
       }
-      float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      if (!pooled) mx *= sc;   // exact tiles: raw scores, base-2 scale applied here
-      // the row max over both halves: exchange with the other warpgroup's thread of this row
-      sm.xmax[bsel][wg][r] = mx;
-      mbar_arrive(&sm.xbar[bsel]);
-      if (!mbar_wait(&sm.xbar[bsel], (t >> 1) & 1, abort)) {
-        ok = false;
-        break;
-      }
-      mx = fmaxf(mx, sm.xmax[bsel][1 - wg][r]);
       const float m_new = fmaxf(m_ref, mx);
       const bool upd = m_new > m_ref + 8.0f;
       const float m_use = upd ? m_new : m_ref;
@@ -471,50 +498,64 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float2 rsa = unf2(add2(rs2[0], rs2[1]));
       l = l * alpha + (rsa.x + rsa.y);
-      // P buffer (t & 1) was last read by P V of tile t - 2; O must be quiet before rescaling
-      if (t > 0 && !mbar_wait(&sm.pvdone, (t - 1) & 1, abort)) {
+      // O_w must be quiet (P V of tile t - 1 done) before it is rescaled
+      if (t > 0 && !mbar_wait(&sm.pvdone[wg], (t - 1) & 1, abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      tmem_st32_at<0>(lane_addr + kColP + 64 * bsel + 32 * wg, pk);
+      if (!(single && wg == 1)) tmem_st32_at<0>(s_addr, pk);   // P over this half's S columns
       // tcgen05.ld / st are warp-collective: the warp rescales if any of its rows needs it
       const bool need = upd && t > 0 && m_ref != -INFINITY;
       if (__any_sync(0xffffffffu, need)) {
         const float f = need ? alpha : 1.f;
-        uint32_t o[64];
-        const uint32_t o_addr = lane_addr + kColO + 64 * wg;
-        tmem_ld32_at<0>(o_addr, o);
-        tmem_ld32_at<32>(o_addr + 32, o);
-        tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-        tmem_st32_at<0>(o_addr, o);
-        tmem_st32_at<32>(o_addr + 32, o);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[64];
+          tmem_ld32_at<0>(o_addr + 64 * half, o);
+          tmem_ld32_at<32>(o_addr + 64 * half + 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+          tmem_st32_at<0>(o_addr + 64 * half, o);
+          tmem_st32_at<32>(o_addr + 64 * half + 32, o);
+        }
       }
       m_ref = m_use;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sm.pready);
+      mbar_arrive(&sm.pready[wg]);
       if (d.flags & 0x100u) break;
     }
-    if (ok && !mbar_wait(&sm.pvdone, t & 1, abort)) ok = false;
-    if (!ok) set_timeout(p.status);
-    tc_fence_after();
-    // combine the two halves' row sums (the max-exchange buffer of the other S parity is free: both
-    // warpgroups read it, for tile t - 1, before arriving at the exchange of tile t)
+    if (ok && !mbar_wait(&sm.pvdone[wg], t & 1, abort)) ok = false;
+    // exchange (m, l) with the other warpgroup's thread of this row, then merge the two halves:
+    // o = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)), M = max(m_0, m_1)
+    float w_self = 0.f, w_other = 0.f, l_tot = 1.f;
     if (ok) {
-      sm.xmax[(t + 1) & 1][wg][r] = l;
+      sm.xm[wg][r] = m_ref;
+      sm.xl[wg][r] = l;
       mbar_arrive(&sm.lbar);
-      if (mbar_wait(&sm.lbar, 0, abort))
-        l = sm.xmax[(t + 1) & 1][0][r] + sm.xmax[(t + 1) & 1][1][r];
-      else
+      if (mbar_wait(&sm.lbar, 0, abort)) {
+        const float m0 = sm.xm[0][r], m1 = sm.xm[1][r];
+        const float l0 = sm.xl[0][r], l1 = sm.xl[1][r];
+        const float M = fmaxf(m0, m1);
+        const float e0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
+        const float e1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+        w_self = wg ? e1 : e0;
+        w_other = wg ? e0 : e1;
+        l_tot = l0 * e0 + l1 * e1;
+        m_ref = M;   // the merged row's reference (base 2)
+      } else {
         ok = false;
+      }
     }
     if (!ok) set_timeout(p.status);
+    tc_fence_after();
     if (__all_sync(0xffffffffu, ok)) {
-      // epilogue: o = O / l (Sol-Attn2: merged with the anchor's complementary tail)
-      float scale_o = 1.f / l;
+      // epilogue: this warpgroup writes output columns 64 wg .. 64 wg + 63 from both accumulators
+      const bool other_written = wg == 1 || o1_written;   // O_1 exists unless only 64-key tiles ran
+      const bool self_written = wg == 0 || o1_written;
+      float scale_o = 1.f / l_tot;
       float tail_w = 0.f;
       const float* nu = nullptr;
       if (kSol2 && row_valid) {
@@ -545,17 +586,23 @@ __global__ void __launch_bounds__(384, 1)
           const float M = fmaxf(m_ref, lz2);
           const float eo = ex2(m_ref - M);
           tail_w = ex2(lz2 - M);
-          const float den = l * eo + tail_w;
+          const float den = l_tot * eo + tail_w;
           scale_o = eo / den;
           tail_w = tail_w / den;
           nu = p.tail_nu + abase * 128 + 64 * wg;
         }
       }
-      uint32_t o[64];
-      const uint32_t o_addr = lane_addr + kColO + 64 * wg;
-      tmem_ld32_at<0>(o_addr, o);
-      tmem_ld32_at<32>(o_addr + 32, o);
+      // O_self columns 64 wg.. and O_other columns 64 wg.. (the other accumulator's same columns)
+      uint32_t oa[64], ob[64];
+      const uint32_t self_addr = lane_addr + kColO + 128 * wg + 64 * wg;
+      const uint32_t other_addr = lane_addr + kColO + 128 * (1 - wg) + 64 * wg;
+      tmem_ld32_at<0>(self_addr, oa);
+      tmem_ld32_at<32>(self_addr + 32, oa);
+      tmem_ld32_at<0>(other_addr, ob);
+      tmem_ld32_at<32>(other_addr + 32, ob);
       tmem_ld_wait();
+      const float ws = (self_written && w_self > 0.f) ? w_self * scale_o : 0.f;
+      const float wo = (other_written && w_other > 0.f) ? w_other * scale_o : 0.f;
       if (row_valid) {
         __nv_bfloat16* orow = p.out + ((size_t)((size_t)b * p.N + tok) * p.H + h) * 128 + 64 * wg;
 #pragma unroll
@@ -564,8 +611,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 8 * c8 + 2 * e;
-            float a0 = __uint_as_float(o[c]) * scale_o;
-            float a1 = __uint_as_float(o[c + 1]) * scale_o;
+            float a0 = ws > 0.f ? __uint_as_float(oa[c]) * ws : 0.f;
+            float a1 = ws > 0.f ? __uint_as_float(oa[c + 1]) * ws : 0.f;
+            if (wo > 0.f) {
+              a0 = fmaf(__uint_as_float(ob[c]), wo, a0);
+              a1 = fmaf(__uint_as_float(ob[c + 1]), wo, a1);
+            }
             if (kSol2 && nu) {
               a0 = fmaf(tail_w, nu[c], a0);
               a1 = fmaf(tail_w, nu[c + 1], a1);
