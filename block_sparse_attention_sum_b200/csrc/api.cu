@@ -217,7 +217,7 @@ int check_launch(const char* what) {
 // Routing prefix shared by all entry points: summaries, threshold statistics, thresholds, bitmask.
 int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                 const Shape& s, const Work& w, float tau, int sink_start, int sink_tokens, bool anchors,
-                cudaStream_t st, int* launches) {
+                bool diag, cudaStream_t st, int* launches) {
   int sb0, sb1;
   sink_blocks(s.N, sink_start, sink_tokens, &sb0, &sb1);
   const unsigned long long init[3] = {0ull, ~0ull, 0ull};
@@ -230,17 +230,30 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   ww.stats = d.stats;
   launch_summary(q, k, v, s, ww, anchors, st);
   launch_kstats(s, ww, st);
-  launch_thresh(s, ww, tau, st);
+  launch_thresh(s, ww, tau, diag, st);
   launch_route(s, ww, sb0, sb1, st);
   *launches += 6;
   d.last_total_pairs = (long long)s.BH * s.Nb * s.Nb;
   return check_launch("routing kernels");
 }
 
+int check_options(const sol_attn_options* o, bool* diag) {
+  *diag = false;
+  if (!o) return SOL_OK;
+  for (int r : o->reserved)
+    if (r != 0) return fail(SOL_ERR_OPTION, "reserved option fields must be zero");
+  if (o->thresh_type != SOL_THRESH_EXACT && o->thresh_type != SOL_THRESH_DIAG)
+    return fail(SOL_ERR_OPTION, "unknown thresh_type %d", o->thresh_type);
+  *diag = o->thresh_type == SOL_THRESH_DIAG;
+  return SOL_OK;
+}
+
 int forward(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau, int sink_start,
-            int sink_tokens, void* stream, bool sol2) {
+            int sink_tokens, const sol_attn_options* opts, void* stream, bool sol2) {
   int rc = validate(q, k, v, out, true, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
+  bool diag;
+  if ((rc = check_options(opts, &diag))) return rc;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;
   int dev;
@@ -264,7 +277,7 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   const auto* qh = static_cast<const __nv_bfloat16*>(q);
   const auto* kh = static_cast<const __nv_bfloat16*>(k);
   const auto* vh = static_cast<const __nv_bfloat16*>(v);
-  if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, st, &launches))) return rc;
+  if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, diag, st, &launches))) return rc;
   if (sol2) {
     launch_groups(qh, kh, vh, s, w, st);
     launch_anchor_tail(s, w, st);
@@ -319,13 +332,25 @@ extern "C" {
 int sol_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
                  int sink_start, int sink_tokens, void* stream) {
   g_err[0] = 0;
-  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, stream, false);
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, nullptr, stream, false);
 }
 
 int sol_attn2_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
                   int sink_start, int sink_tokens, void* stream) {
   g_err[0] = 0;
-  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, stream, true);
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, nullptr, stream, true);
+}
+
+int sol_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                    int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream) {
+  g_err[0] = 0;
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, opts, stream, false);
+}
+
+int sol_attn2_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                     int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream) {
+  g_err[0] = 0;
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, opts, stream, true);
 }
 
 const char* sol_attn_last_error(void) { return g_err; }
@@ -347,11 +372,14 @@ int sol_attn_get_device_status(void* stream) {
   return SOL_OK;
 }
 
-int sol_attn_debug_route(const void* q, const void* k, int B, int N, int H, float tau, int sink_start,
-                         int sink_tokens, unsigned char* mask, float* thresh, void* stream) {
+int sol_attn_debug_route_ex(const void* q, const void* k, int B, int N, int H, float tau, int sink_start,
+                            int sink_tokens, const sol_attn_options* opts, unsigned char* mask, float* thresh,
+                            void* stream) {
   g_err[0] = 0;
   int rc = validate(q, k, nullptr, nullptr, false, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
+  bool diag;
+  if ((rc = check_options(opts, &diag))) return rc;
   if (!mask) return fail(SOL_ERR_NULL, "mask must be non-NULL");
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;
@@ -367,7 +395,7 @@ int sol_attn_debug_route(const void* q, const void* k, int B, int N, int H, floa
   int launches = 0;
   // the summary kernel reads v as well; pass k, whose summaries are simply discarded
   if ((rc = run_routing(*d, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                        static_cast<const __nv_bfloat16*>(k), s, w, tau, sink_start, sink_tokens, false, st,
+                        static_cast<const __nv_bfloat16*>(k), s, w, tau, sink_start, sink_tokens, false, diag, st,
                         &launches)))
     return rc;
   launch_expand_mask(s, w, mask, st);
@@ -378,6 +406,11 @@ int sol_attn_debug_route(const void* q, const void* k, int B, int N, int H, floa
   d->last_launches = launches + 1;
   g_last_device = dev;
   return SOL_OK;
+}
+
+int sol_attn_debug_route(const void* q, const void* k, int B, int N, int H, float tau, int sink_start,
+                         int sink_tokens, unsigned char* mask, float* thresh, void* stream) {
+  return sol_attn_debug_route_ex(q, k, B, N, H, tau, sink_start, sink_tokens, nullptr, mask, thresh, stream);
 }
 
 int sol_attn_last_stats(long long* exact_pairs, long long* total_pairs, int* min_row, int* max_row) {

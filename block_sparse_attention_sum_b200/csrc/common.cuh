@@ -65,7 +65,7 @@ void set_last_error(const char* msg);
 void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
                     const Work& w, bool anchors, cudaStream_t st);
 void launch_kstats(const Shape& s, const Work& w, cudaStream_t st);
-void launch_thresh(const Shape& s, const Work& w, float tau, cudaStream_t st);
+void launch_thresh(const Shape& s, const Work& w, float tau, bool diag, cudaStream_t st);
 void launch_route(const Shape& s, const Work& w, int sink_b0, int sink_b1, cudaStream_t st);
 void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, cudaStream_t st);
 

@@ -192,7 +192,7 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   const auto* vh = static_cast<const __nv_bfloat16*>(v);
   launch_summary(qh, kh, vh, s, w, false, st);
   launch_kstats(s, w, st);
-  launch_thresh(s, w, tau, st);
+  launch_thresh(s, w, tau, false, st);
   launch_route(s, w, sb0, sb1, st);
   FwdParams p{};
   p.N = N;

@@ -195,7 +195,7 @@ __global__ void kgram_reduce_kernel(Shape s, Work w, const float* partial) {
 // -------------------------------------------------------------------------------------------------
 constexpr int kThreshPad = 68;
 
-__global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau) {
+__global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau, int diag) {
   extern __shared__ __align__(16) float tsm[];
   float* cov_s = tsm;                                // [128][128]
   float* qt = tsm + kHeadDim * kHeadDim;             // [128][68]  Qbar^T of the 64 rows
@@ -217,6 +217,18 @@ __global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau)
     for (int c = 0; c < kHeadDim; ++c) m += (double)qt[c * kThreshPad + tid] * mk[c];
     mu_s[tid] = (float)m;
   }
+  if (diag) {
+    // diagonal estimator: sigma_i^2 = s^2 sum_c Qbar_ic^2 C_cc
+    if (tid < 64) {
+      float q = 0.f;
+      for (int c = 0; c < kHeadDim; ++c) {
+        const float x = qt[c * kThreshPad + tid];
+        q = fmaf(x * x, cov_s[c * kHeadDim + c], q);
+      }
+      part[tid][0] = q;
+      for (int c = 1; c < 16; ++c) part[tid][c] = 0.f;
+    }
+  } else {
   const int ti = tid >> 4, tj = tid & 15;   // rows 4 ti .. 4 ti + 3, columns 8 tj .. 8 tj + 7
   float y[4][8];
 #pragma unroll
@@ -241,6 +253,7 @@ __global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau)
 #pragma unroll
     for (int c = 0; c < 8; ++c) q = fmaf(qt[(8 * tj + c) * kThreshPad + 4 * ti + a], y[a][c], q);
     part[4 * ti + a][tj] = q;
+  }
   }
   __syncthreads();
   if (tid < 64 && i0 + tid < s.Nb) {
@@ -272,9 +285,29 @@ __global__ void __launch_bounds__(128) route_kernel(Shape s, Work w, int sink_b0
   const int ti = tid >> 4, tj = tid & 15;           // rows 8 ti .. 8 ti + 7, columns 8 tj .. 8 tj + 7
   const float* qb = w.qbar + (size_t)bh * s.Nb * kHeadDim;
   const float* kb = w.kbar + (size_t)bh * s.Nb * kHeadDim;
-  for (int idx = tid; idx < kRouteRows * kHeadDim; idx += 128) {
-    const int r = idx / kHeadDim, c = idx % kHeadDim;
-    Qt[c * kRoutePadQ + r] = (i0 + r < s.Nb) ? qb[(size_t)(i0 + r) * kHeadDim + c] : 0.f;
+  {
+    // thread = (row, half of the channels); 16-byte loads, eight in flight; the transposed stores
+    // of a warp hit 32 consecutive rows (no bank conflicts)
+    const int row = tid & 63, c0 = (tid >> 6) * 64;
+    const bool in = i0 + row < s.Nb;
+    const float4* src = reinterpret_cast<const float4*>(qb + (size_t)(i0 + row) * kHeadDim + c0);
+#pragma unroll
+    for (int k0 = 0; k0 < 16; k0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (in) v[k] = __ldg(src + k0 + k);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int c = c0 + 4 * (k0 + k);
+        Qt[(c + 0) * kRoutePadQ + row] = v[k].x;
+        Qt[(c + 1) * kRoutePadQ + row] = v[k].y;
+        Qt[(c + 2) * kRoutePadQ + row] = v[k].z;
+        Qt[(c + 3) * kRoutePadQ + row] = v[k].w;
+      }
+    }
   }
   if (tid < kRouteRows) {
     th[tid] = (i0 + tid < s.Nb) ? w.thresh[(size_t)bh * s.Nb + i0 + tid] : 0.f;
@@ -282,9 +315,28 @@ __global__ void __launch_bounds__(128) route_kernel(Shape s, Work w, int sink_b0
   }
   for (int j0 = 0; j0 < s.Nb; j0 += kRouteCols) {
     __syncthreads();
-    for (int idx = tid; idx < kRouteCols * kHeadDim; idx += 128) {
-      const int r = idx / kHeadDim, c = idx % kHeadDim;
-      Kt[c * kRoutePadK + r] = (j0 + r < s.Nb) ? kb[(size_t)(j0 + r) * kHeadDim + c] : 0.f;
+    {
+      // thread = key block row; 16-byte loads, eight in flight; conflict-free transposed stores
+      const int row = tid;
+      const bool in = j0 + row < s.Nb;
+      const float4* src = reinterpret_cast<const float4*>(kb + (size_t)(j0 + row) * kHeadDim);
+#pragma unroll
+      for (int k0 = 0; k0 < 32; k0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (in) v[k] = __ldg(src + k0 + k);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int c = 4 * (k0 + k);
+          Kt[(c + 0) * kRoutePadK + row] = v[k].x;
+          Kt[(c + 1) * kRoutePadK + row] = v[k].y;
+          Kt[(c + 2) * kRoutePadK + row] = v[k].z;
+          Kt[(c + 3) * kRoutePadK + row] = v[k].w;
+        }
+      }
     }
     __syncthreads();
     float acc[8][8];
@@ -368,10 +420,10 @@ void launch_kstats(const Shape& s, const Work& w, cudaStream_t st) {
   kgram_reduce_kernel<<<dim3(kHeadDim * kHeadDim / 256, s.BH), 256, 0, st>>>(s, w, w.gram_partial);
 }
 
-void launch_thresh(const Shape& s, const Work& w, float tau, cudaStream_t st) {
+void launch_thresh(const Shape& s, const Work& w, float tau, bool diag, cudaStream_t st) {
   const int smem = (kHeadDim * kHeadDim + kHeadDim * kThreshPad) * sizeof(float);
   cudaFuncSetAttribute(thresh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  thresh_kernel<<<dim3((s.Nb + 63) / 64, s.BH), 256, smem, st>>>(s, w, tau);
+  thresh_kernel<<<dim3((s.Nb + 63) / 64, s.BH), 256, smem, st>>>(s, w, tau, diag ? 1 : 0);
 }
 
 void launch_route(const Shape& s, const Work& w, int sink_b0, int sink_b1, cudaStream_t st) {

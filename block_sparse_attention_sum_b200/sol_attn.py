@@ -20,6 +20,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.
 EXPORTS = [
     "sol_attn_fwd",
     "sol_attn2_fwd",
+    "sol_attn_fwd_ex",
+    "sol_attn2_fwd_ex",
+    "sol_attn_debug_route_ex",
     "sol_attn_last_error",
     "sol_attn_get_device_status",
     "sol_attn_debug_route",
@@ -35,7 +38,22 @@ EXPORTS = [
 STATUS = {
     0: "SOL_OK", -1: "SOL_ERR_NULL", -2: "SOL_ERR_SHAPE", -3: "SOL_ERR_TAU", -4: "SOL_ERR_SINK",
     -5: "SOL_ERR_ALIGN", -6: "SOL_ERR_ALLOC", -7: "SOL_ERR_LAUNCH", -8: "SOL_ERR_DEVICE", -9: "SOL_ERR_TIMEOUT",
+    -10: "SOL_ERR_OPTION",
 }
+
+THRESH_TYPES = {"exact": 0, "diag": 1}
+
+
+class Options(ctypes.Structure):
+    """sol_attn_options (include/sol_attn.h)."""
+
+    _fields_ = [("thresh_type", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+
+
+def _options(thresh_type: str):
+    if thresh_type not in THRESH_TYPES:
+        raise ValueError(f"thresh_type must be one of {sorted(THRESH_TYPES)}")
+    return Options(THRESH_TYPES[thresh_type])
 
 
 class SolAttnError(RuntimeError):
@@ -62,6 +80,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_fwd.restype = i
     lib.sol_attn2_fwd.argtypes = fwd_args
     lib.sol_attn2_fwd.restype = i
+    op = ctypes.POINTER(Options)
+    ex_args = [vp, vp, vp, vp, i, i, i, f, i, i, op, vp]
+    lib.sol_attn_fwd_ex.argtypes = ex_args
+    lib.sol_attn_fwd_ex.restype = i
+    lib.sol_attn2_fwd_ex.argtypes = ex_args
+    lib.sol_attn2_fwd_ex.restype = i
+    lib.sol_attn_debug_route_ex.argtypes = [vp, vp, i, i, i, f, i, i, op, vp, vp, vp]
+    lib.sol_attn_debug_route_ex.restype = i
     lib.sol_attn_last_error.argtypes = []
     lib.sol_attn_last_error.restype = ctypes.c_char_p
     lib.sol_attn_get_device_status.argtypes = [vp]
@@ -112,28 +138,33 @@ def _check_qkv(q, k, v=None):
     return q.shape[0], q.shape[1], q.shape[2]
 
 
-def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream):
+def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type="exact"):
     B, N, H = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device != q.device:
         raise ValueError("out must be a contiguous BF16 tensor shaped like q")
     lib = load_library()
+    args = [q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, float(tau), int(sink_start),
+            int(sink_tokens)]
     with torch.cuda.device(q.device):
-        rc = getattr(lib, fn_name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H,
-                                   float(tau), int(sink_start), int(sink_tokens), _stream_handle(stream))
+        if thresh_type != "exact":
+            opts = _options(thresh_type)
+            rc = getattr(lib, fn_name + "_ex")(*args, ctypes.byref(opts), _stream_handle(stream))
+        else:
+            rc = getattr(lib, fn_name)(*args, _stream_handle(stream))
     _check(rc)
     return out
 
 
-def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
+def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact"):
     """Sol-Attn forward through the C ABI; returns ``out`` (BF16 [B, N, H, 128])."""
-    return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream)
+    return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type)
 
 
-def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
+def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact"):
     """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
-    return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream)
+    return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type)
 
 
 def sol_attn_fwd_noalloc(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
@@ -152,7 +183,7 @@ def sol_attn2(q, k, v, tau=1.0, sink_start=None, sink_tokens=0, out=None):
     return sol_attn2_fwd(q, k, v, tau, -1 if sink_start is None else sink_start, sink_tokens, out)
 
 
-def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None):
+def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None, thresh_type="exact"):
     """Exact-block mask (uint8 [B, H, Nb, Nb]) and thresholds (float32 [B, H, Nb]) from the GPU router."""
     B, N, H = _check_qkv(q, k)
     Nb = math.ceil(N / BLOCK)
@@ -160,8 +191,10 @@ def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None):
     thresh = torch.empty(B, H, Nb, dtype=torch.float32, device=q.device)
     lib = load_library()
     with torch.cuda.device(q.device):
-        rc = lib.sol_attn_debug_route(q.data_ptr(), k.data_ptr(), B, N, H, float(tau), int(sink_start),
-                                      int(sink_tokens), mask.data_ptr(), thresh.data_ptr(), _stream_handle(stream))
+        opts = _options(thresh_type)
+        rc = lib.sol_attn_debug_route_ex(q.data_ptr(), k.data_ptr(), B, N, H, float(tau), int(sink_start),
+                                         int(sink_tokens), ctypes.byref(opts), mask.data_ptr(), thresh.data_ptr(),
+                                         _stream_handle(stream))
     _check(rc)
     return mask, thresh
 

@@ -52,8 +52,21 @@ typedef enum {
   SOL_ERR_ALLOC = -6,   /* workspace allocation failed */
   SOL_ERR_LAUNCH = -7,  /* a CUDA launch or runtime call failed */
   SOL_ERR_DEVICE = -8,  /* no usable sm_100 device */
-  SOL_ERR_TIMEOUT = -9  /* a bounded wait inside a kernel ran out (see sol_attn_get_device_status) */
+  SOL_ERR_TIMEOUT = -9, /* a bounded wait inside a kernel ran out (see sol_attn_get_device_status) */
+  SOL_ERR_OPTION = -10  /* an option value is out of range or a reserved field is nonzero */
 } sol_status;
+
+/* Threshold estimators ("Sol-Attn" paper: Eq. (5) and appendix "Diagonal threshold estimator"). */
+typedef enum {
+  SOL_THRESH_EXACT = 0, /* full-covariance sigma_i (the Sol-Attn README default, thresh_type="exact") */
+  SOL_THRESH_DIAG = 1   /* sigma_i^2 = (Qbar_i * Qbar_i) . v_K with v_K the per-channel variance of Kbar */
+} sol_thresh_type;
+
+/* Options of the _ex entry points.  A NULL pointer means all defaults; reserved fields must be 0. */
+typedef struct {
+  int thresh_type;   /* sol_thresh_type */
+  int reserved[7];
+} sol_attn_options;
 
 /*
  * Sol-Attn forward (arXiv 2607.24027, sections 3.1-3.2).  For each (b, h) and 64-token query
@@ -80,6 +93,20 @@ int sol_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, 
  */
 int sol_attn2_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
                   int sink_start, int sink_tokens, void* stream);
+
+/*
+ * sol_attn_fwd / sol_attn2_fwd / sol_attn_debug_route with options (`opts` may be NULL).  With
+ * SOL_THRESH_DIAG the threshold's variance keeps only the diagonal of the key-block-mean covariance
+ * (the mean mu_i stays exact); everything else is as in the plain entry points.  An invalid option
+ * returns SOL_ERR_OPTION before anything is launched.
+ */
+int sol_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                    int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream);
+int sol_attn2_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                     int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream);
+int sol_attn_debug_route_ex(const void* q, const void* k, int B, int N, int H, float tau, int sink_start,
+                            int sink_tokens, const sol_attn_options* opts, unsigned char* mask, float* thresh,
+                            void* stream);
 
 /* Message for the last error returned on the calling thread ("" if none).  Owned by the library. */
 const char* sol_attn_last_error(void);

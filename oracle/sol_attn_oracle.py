@@ -35,7 +35,8 @@ R1  Scale: s = 1/sqrt(128) on token logits, proxies, thresholds and surrogate lo
 R2  "N" in Eq. (5) is the number of key blocks Nb; every block, the partial last one included,
     has equal weight in mu_i and sigma_i.
 R3  Threshold type "exact" (full covariance), the README default; evaluated here by its
-    definition (mean and variance of the proxy row), which Eq. (5) restates.
+    definition (mean and variance of the proxy row), which Eq. (5) restates.  Type "diag" follows
+    the appendix's diagonal estimator (exact mean, diagonal of the key-mean covariance).
 R4  Ties s_ij == tau_i are not exact (strict ">", Eq. (4)).
 R5  Adjacent blocks: key blocks j with |i - j| <= 1 are always exact ([sdcpp]).
 R6  Partial last block: means over its valid tokens, surrogate mass n_j (its token count).
@@ -144,6 +145,19 @@ def threshold(shat: np.ndarray, tau: float):
     return mu, sigma, mu + tau * sigma
 
 
+def threshold_diag(Qbar: np.ndarray, Kbar: np.ndarray, tau: float):
+    """Diagonal threshold estimator (appendix "Diagonal threshold estimator"): the mean mu_i is
+    exact; the variance keeps only the diagonal of the key-mean covariance,
+    v_K = mean_j Kbar_j * Kbar_j - mu_K * mu_K and sigma_i^2 = (Qbar_i * Qbar_i) . v_K (scaled by s^2,
+    reading R1).  Returns mu, sigma, tau_i = mu_i + tau * sigma_i."""
+    Nb = Kbar.shape[0]
+    muK = Kbar.sum(axis=0) / Nb
+    vK = (Kbar * Kbar).sum(axis=0) / Nb - muK * muK
+    mu = SCALE * (Qbar @ muK)
+    sigma = SCALE * np.sqrt(np.maximum((Qbar * Qbar) @ vK, 0.0))
+    return mu, sigma, mu + tau * sigma
+
+
 def sink_block_flags(N: int, sink_start: int, sink_tokens: int) -> np.ndarray:
     """Key blocks that overlap the exact sink range (README "Exact KV sink"; reading R8)."""
     Nb = num_blocks(N)
@@ -207,22 +221,25 @@ def sol_attn_rows(q_rows, k_bh, v_bh, mask_row, Kbar, Vhat, counts):
     return num / den[:, None]
 
 
-def _routing_for_head(q_bh, k_bh, tau, sink_flags):
+def _routing_for_head(q_bh, k_bh, tau, sink_flags, thresh_type="exact"):
     N = q_bh.shape[0]
     Qbar = block_means(q_bh)
     Kbar = block_means(k_bh)
     shat = proxy_scores(Qbar, Kbar)
-    mu, sigma, thresh = threshold(shat, tau)
+    if thresh_type == "diag":
+        mu, sigma, thresh = threshold_diag(Qbar, Kbar, tau)
+    else:
+        mu, sigma, thresh = threshold(shat, tau)
     mask = exact_mask(shat, thresh, sink_flags)
     return dict(Qbar=Qbar, Kbar=Kbar, shat=shat, mu=mu, sigma=sigma, thresh=thresh, mask=mask,
                 counts=block_counts(N))
 
 
-def routing(q, k, tau: float, sink_start: int = -1, sink_tokens: int = 0):
+def routing(q, k, tau: float, sink_start: int = -1, sink_tokens: int = 0, thresh_type: str = "exact"):
     """Per (b, h): proxies, mu, sigma, thresholds and exact masks. Returns a dict of stacked arrays."""
     B, N, H, _ = q.shape
     sink = sink_block_flags(N, sink_start, sink_tokens)
-    per = [[_routing_for_head(head_slice(q, b, h), head_slice(k, b, h), tau, sink) for h in range(H)]
+    per = [[_routing_for_head(head_slice(q, b, h), head_slice(k, b, h), tau, sink, thresh_type) for h in range(H)]
            for b in range(B)]
     keys = ["shat", "mu", "sigma", "thresh", "mask"]
     return {key: np.stack([np.stack([per[b][h][key] for h in range(H)]) for b in range(B)]) for key in keys}
@@ -233,7 +250,8 @@ def _row_subset(N, qblocks):
     return range(Nb) if qblocks is None else qblocks
 
 
-def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None):
+def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None,
+             thresh_type: str = "exact"):
     """Sol-Attn forward. Returns dict with ``out`` (FP64 [B, N, H, 128]; NaN for rows not computed),
     ``mask`` [B, H, Nb, Nb], ``shat``, ``thresh``.
 
@@ -250,7 +268,7 @@ def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qb
     pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
     for b, h in pairs:
         q_bh, k_bh, v_bh = head_slice(q, b, h), head_slice(k, b, h), head_slice(v, b, h)
-        r = _routing_for_head(q_bh, k_bh, tau, sink)
+        r = _routing_for_head(q_bh, k_bh, tau, sink, thresh_type)
         Vhat = block_sums(v_bh)
         masks[b, h], shats[b, h], threshs[b, h] = r["mask"], r["shat"], r["thresh"]
         for i in _row_subset(N, qblocks):

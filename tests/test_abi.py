@@ -58,3 +58,12 @@ def test_no_device_is_an_error_not_a_fallback(lib):
         pytest.skip("a GPU is present")
     rc = _fwd(lib)
     assert rc == -8, rc
+
+
+def test_invalid_options_are_rejected_on_the_host(lib):
+    opts = sa.Options(7)
+    rc = lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None)
+    assert rc == -10
+    opts = sa.Options(1)
+    opts.reserved[3] = 1
+    assert lib.sol_attn2_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10

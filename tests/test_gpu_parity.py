@@ -151,3 +151,24 @@ def test_stream_and_stats_and_timing():
     exact, total, mn, mx = sa.last_stats()
     assert total == 2 * 32 * 32 and 0 < exact <= total and 2 <= mn <= mx <= 32
     assert sa.last_launch_count() == 7
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan"])
+def test_diagonal_threshold_estimator(name):
+    """thresh_type="diag" (appendix "Diagonal threshold estimator") against the oracle."""
+    w = WORKLOADS[name]
+    q, k, v = w.make_inputs("cpu")
+    tau = w.resolved_tau()
+    ref = orc.sol_attn(q, k, v, tau, w.sink_start, w.sink_tokens, thresh_type="diag")
+    full = orc.routing(q, k, tau, w.sink_start, w.sink_tokens, thresh_type="diag")
+    ref.update(shat=full["shat"], thresh=full["thresh"])
+    qd, kd, vd = _to_gpu(q, k, v)
+    out = sa.sol_attn_fwd(qd, kd, vd, tau, w.sink_start, w.sink_tokens, thresh_type="diag")
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    gmask, gthr = sa.debug_route(qd, kd, tau, w.sink_start, w.sink_tokens, thresh_type="diag")
+    skip = check_mask(gmask.cpu().numpy(), ref)
+    np.testing.assert_allclose(gthr.cpu().numpy(), full["thresh"], rtol=1e-5, atol=2e-6)
+    compare_outputs(out.float().cpu().numpy(), ref["out"], w.N, skip_rows=skip)
+    exact = orc.routing(q, k, tau, w.sink_start, w.sink_tokens)
+    assert not np.array_equal(exact["mask"], full["mask"])   # the estimator changes the routing

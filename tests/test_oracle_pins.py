@@ -267,3 +267,40 @@ def test_surrogate_reduces_error_against_dense():
     rel = lambda x: np.linalg.norm(x - dense) / np.linalg.norm(dense)
     assert orc.realised_sparsity(r["mask"]) > 0.5
     assert rel(r["out"]) < rel(exact_only)
+
+
+# ------------------------------------------------------------- diagonal threshold estimator
+
+def test_diagonal_estimator_equals_exact_when_key_covariance_is_diagonal():
+    """Appendix "Diagonal threshold estimator": with key-block means whose centred deviations have
+    orthogonal channel columns, the covariance is diagonal and the estimator is exact."""
+    g = np.random.default_rng(31)
+    Nb = 160
+    U, _ = np.linalg.qr(g.standard_normal((Nb, D)))          # orthonormal columns
+    U -= U.mean(axis=0)                                       # centre ...
+    U, _ = np.linalg.qr(U)                                    # ... and re-orthonormalise
+    assert np.abs(U.mean(axis=0)).max() < 1e-12
+    Kbar = 0.7 + U * g.uniform(0.5, 3.0, D)[None, :]
+    Qbar = g.standard_normal((40, D))
+    mu_e, sig_e, thr_e = orc.threshold(orc.proxy_scores(Qbar, Kbar), 1.1)
+    mu_d, sig_d, thr_d = orc.threshold_diag(Qbar, Kbar, 1.1)
+    np.testing.assert_allclose(mu_d, mu_e, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(sig_d, sig_e, rtol=1e-9)
+    np.testing.assert_allclose(thr_d, thr_e, rtol=1e-9, atol=1e-12)
+
+
+def test_diagonal_estimator_drops_channel_correlation():
+    """With perfectly correlated channels the diagonal variance differs from the exact one by the
+    off-diagonal terms, and equals the hand-computed sum of per-channel variances."""
+    Nb = 50
+    a = np.linspace(-1, 1, Nb)
+    Kbar = np.zeros((Nb, D))
+    Kbar[:, 0] = a
+    Kbar[:, 1] = a                                            # channel 1 copies channel 0
+    Qbar = np.zeros((1, D))
+    Qbar[0, 0] = Qbar[0, 1] = 1.0
+    _, sig_d, _ = orc.threshold_diag(Qbar, Kbar, 0.0)
+    _, sig_e, _ = orc.threshold(orc.proxy_scores(Qbar, Kbar), 0.0)
+    va = a.var()
+    assert sig_d[0] == pytest.approx(S * np.sqrt(2 * va), rel=1e-12)
+    assert sig_e[0] == pytest.approx(S * np.sqrt(4 * va), rel=1e-12)
