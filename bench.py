@@ -40,11 +40,51 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="s64k")
-    ap.add_argument("--cpu-sample-blocks", type=int, default=24,
-                    help="query blocks of one head the CPU oracle baseline evaluates")
+    ap.add_argument("--cpu-sample-heads", type=int, default=2,
+                    help="heads (all query blocks each) the CPU oracle baseline evaluates")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
+
+
+def rank_seed(workload, rank: int) -> int:
+    """Seed of a rank's inputs: every rank runs its own batch element (weak scaling, no exchange)."""
+    return workload.seed + 100 * rank
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of a list of floats over all ranks (the timing rule: slowest rank counts)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "attn_fwd_dram_traffic.json")
+KERNEL_SOURCE = os.path.join(ROOT, "block_sparse_attention_sum_b200", "csrc", "attn_fwd.cu")
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def measured_traffic(workload_name: str):
+    """DRAM bytes per launch of the fused kernel from a committed ncu capture, if that capture was
+    taken on this workload with the current kernel source (else None)."""
+    if not os.path.exists(TRAFFIC_PATH):
+        return None
+    with open(TRAFFIC_PATH) as f:
+        rec = json.load(f)
+    entry = rec.get(workload_name)
+    if not entry or entry.get("source_sha256") != kernel_source_digest():
+        return None
+    return entry["dram_bytes_per_launch"]
 
 
 def load_peaks():
@@ -118,9 +158,10 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------------ CPU baseline
 
-def cpu_baseline(workload, n_blocks: int, q=None, k=None, v=None):
-    """The FP64 oracle, as it stands, on one head: full summaries / thresholds for that head and
-    ``n_blocks`` seeded query blocks.  Returns the oracle's effective TFLOP/s on that sample."""
+def cpu_baseline(workload, heads, n_blocks: int, q=None, k=None, v=None, block_seed: int = 7):
+    """The FP64 oracle, as it stands, on a bounded sample of the workload: for each (b, h) in
+    ``heads`` its summaries and thresholds in full and ``n_blocks`` seeded query blocks (all of them
+    if ``n_blocks`` >= Nb).  Returns the oracle's effective TFLOP/s on that sample."""
     import numpy as np
     from threadpoolctl import threadpool_info
 
@@ -130,20 +171,25 @@ def cpu_baseline(workload, n_blocks: int, q=None, k=None, v=None):
         q, k, v = workload.make_inputs("cpu")
     tau = workload.resolved_tau()
     Nb = orc.num_blocks(workload.N)
-    blocks = sorted(np.random.default_rng(7).choice(Nb, size=min(n_blocks, Nb), replace=False).tolist())
+    if n_blocks >= Nb:
+        blocks = list(range(Nb))
+    else:
+        blocks = sorted(np.random.default_rng(block_seed).choice(Nb, size=n_blocks, replace=False).tolist())
     fn = getattr(orc, workload.entry)
     t0 = time.perf_counter()
-    r = fn(q, k, v, tau, workload.sink_start, workload.sink_tokens, qblocks=blocks, heads=[(0, 0)])
+    r = fn(q, k, v, tau, workload.sink_start, workload.sink_tokens, qblocks=blocks, heads=heads)
     dt = time.perf_counter() - t0
-    rows = r["mask"][0, 0][blocks]
-    exact = int(rows.sum())
-    total = rows.size
+    exact = total = 0
+    for b, h in heads:
+        rows = r["mask"][b, h][blocks]
+        exact += int(rows.sum())
+        total += rows.size
     flops, _ = effective_flops(1, workload.N, 1, exact, total)
     threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{workload.name}: head 0 of {workload.H}, {len(blocks)} of {Nb} query blocks "
-                      f"(summaries and thresholds of that head in full), FP64 numpy, {dt:.1f} s",
-            "seconds": dt}
+            "sample": f"{workload.name}: {len(heads)} of {workload.B * workload.H} heads, {len(blocks)} of {Nb} "
+                      f"query blocks each (their summaries and thresholds in full), FP64 numpy, {dt:.1f} s",
+            "seconds": dt, "flops": flops}
 
 
 # ---------------------------------------------------------------------------------------------- main
@@ -161,16 +207,28 @@ def main():
         raise SystemExit("--warmup must be >= 3")
 
     if args.impl == "reference":
+        # the reference arm is the FP64 oracle: each step is one head with 64 seeded query blocks
         if rank != 0:
             return 0
-        base = cpu_baseline(w, args.cpu_sample_blocks)
-        line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": "TFLOP/s", "n_gpus": args.gpus,
-                "steps": 1, "warmup": 0, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "seq_len": w.N,
-                           "global_batch": w.B, "parallelism": "cpu"},
-                "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
-                "e2e": {"value": base["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        q, k, v = w.make_inputs("cpu")
+        flops = secs = 0.0
+        base = None
+        for i in range(args.warmup + args.steps):
+            head = (0, i % w.H)
+            base = cpu_baseline(w, [head], 64, q, k, v, block_seed=i)
+            if i >= args.warmup:
+                flops += base["flops"]
+                secs += base["seconds"]
+        value = flops / secs / 1e12
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "seq_len": w.N, "global_batch": w.B,
+                           "parallelism": "cpu"},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": base["cores"], "kind": "oracle",
+                                 "sample": f"{w.name}: per step one head (cycling), 64 seeded query blocks, "
+                                           "its summaries and thresholds in full; FP64 numpy"},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
 
@@ -187,7 +245,7 @@ def main():
     # inputs: seeded on the CPU (deterministic), pinned for the end-to-end leg; each rank its own batch element
     from block_sparse_attention_sum_b200.inputs import grf_qkv, iid_qkv
 
-    seed = w.seed + 100 * rank
+    seed = rank_seed(w, rank)
     if w.kind == "grf":
         qh, kh, vh = grf_qkv(w.B, w.H, w.grid, seed_base=seed)
     else:
@@ -231,10 +289,7 @@ def main():
     sa.set_kernel_timing(False)
     assert sa.get_device_status() == 0, "device status after the timed region"
 
-    t = torch.tensor([elapsed_ms, kernel_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, kernel_ms = float(t[0]), float(t[1])
+    elapsed_ms, kernel_ms = max_over_ranks([elapsed_ms, kernel_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
     flops_step, exact_flops_step = effective_flops(w.B, w.N, w.H, exact, total)
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
@@ -263,10 +318,7 @@ def main():
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        t2 = torch.tensor([a.elapsed_time(b) / e2e_steps], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t2[0])
+        e2e_ms = max_over_ranks([a.elapsed_time(b) / e2e_steps], world, dev)[0]
         e2e = {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 3 * qh.numel() * qh.element_size(),
                "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": e2e_steps}
@@ -276,7 +328,7 @@ def main():
     peak_burst = float(peaks["bf16_tflops"])
     achieved = flops_step / (kernel_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sust, "unit": "TFLOP/s",
-                "frac": achieved / peak_sust, "traffic": None,
+                "frac": achieved / peak_sust, "traffic": measured_traffic(w.name),
                 "kernel": "attn_fwd_kernel<false> (fused routing + attention)",
                 "kernel_ms": kernel_ms, "peak_kind": f"bf16 dense sustained ({peaks['source']})",
                 "frac_of_burst": achieved / peak_burst}
@@ -295,7 +347,7 @@ def main():
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clock_info}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(w, args.cpu_sample_blocks, qh, kh, vh)
+        cb = cpu_baseline(w, [(0, h) for h in range(args.cpu_sample_heads)], 1 << 30, qh, kh, vh)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
     if rank == 0:
         print(json.dumps(line), flush=True)
