@@ -116,10 +116,11 @@ size_t carve(const Shape& s, bool sol2, char* base, Work* w) {
   if (sol2) {
     const size_t na = (size_t)s.Na;
     t.qanchor = reinterpret_cast<float*>(take(bh * na * d * 4));
+    t.qanchor_h = reinterpret_cast<__nv_bfloat16*>(take(bh * na * d * 2));
     t.qdir = reinterpret_cast<float*>(take(bh * d * 4));
-    t.gk = reinterpret_cast<float*>(take(bh * nb * 2 * d * 4));
-    t.gv = reinterpret_cast<float*>(take(bh * nb * 2 * d * 4));
-    t.gcount = reinterpret_cast<int*>(take(bh * nb * 2 * 4));
+    t.gk_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * 2 * d * 2));
+    t.gv_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * 2 * d * 2));
+    t.glog2n = reinterpret_cast<float*>(take(bh * (size_t)tail_groups_padded(s) * 4));
     t.tail_logz = reinterpret_cast<float*>(take(bh * na * 4));
     t.tail_mu = reinterpret_cast<float*>(take(bh * na * d * 4));
     t.tail_nu = reinterpret_cast<float*>(take(bh * na * d * 4));
@@ -197,16 +198,19 @@ int encode_bthd(CUtensorMap* m, const void* base, const Shape& s) {
   return r == CUDA_SUCCESS ? SOL_OK : fail(SOL_ERR_LAUNCH, "cuTensorMapEncodeTiled (BTHD) failed: %d", (int)r);
 }
 
-int encode_pooled(CUtensorMap* m, const void* base, const Shape& s) {
-  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)s.Nb, (cuuint64_t)s.BH};
-  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)s.Nb * kHeadDim * 2};
+// [BH][rows][128] BF16 rows, 64 x 128 x 1 boxes (pooled block means, anchor means, group means)
+int encode_rows(CUtensorMap* m, const void* base, int rows, const Shape& s) {
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)s.BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)rows * kHeadDim * 2};
   const cuuint32_t box[3] = {64, 128, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? SOL_OK : fail(SOL_ERR_LAUNCH, "cuTensorMapEncodeTiled (pooled) failed: %d", (int)r);
+  return r == CUDA_SUCCESS ? SOL_OK : fail(SOL_ERR_LAUNCH, "cuTensorMapEncodeTiled (rows) failed: %d", (int)r);
 }
+
+int encode_pooled(CUtensorMap* m, const void* base, const Shape& s) { return encode_rows(m, base, s.Nb, s); }
 
 int check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
@@ -279,8 +283,13 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   const auto* vh = static_cast<const __nv_bfloat16*>(v);
   if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, diag, st, &launches))) return rc;
   if (sol2) {
+    CUtensorMap tmaps[3];
+    if ((rc = encode_rows(&tmaps[0], w.qanchor_h, s.Na, s)) || (rc = encode_rows(&tmaps[1], w.gk_h, 2 * s.Nb, s)) ||
+        (rc = encode_rows(&tmaps[2], w.gv_h, 2 * s.Nb, s)))
+      return rc;
     launch_groups(qh, kh, vh, s, w, st);
-    launch_anchor_tail(s, w, st);
+    cudaError_t te = launch_tail_tc(tmaps, s, w, d->status, st);
+    if (te != cudaSuccess) return fail(SOL_ERR_LAUNCH, "Sol-Attn2 tail launch: %s", cudaGetErrorString(te));
     launches += 3;
     if ((rc = check_launch("Sol-Attn2 tail kernels"))) return rc;
   }

@@ -49,10 +49,12 @@ struct Work {
   unsigned long long* stats;  // [0] exact pairs, [1] min row, [2] max row (as unsigned)
   // Sol-Attn2
   float* qanchor;         // [BH][Na][128]  anchor means of Q
+  __nv_bfloat16* qanchor_h;  // [BH][Na][128] BF16 copy (tail MMA operand)
   float* qdir;            // [BH][128]      mean query (the grouping direction)
-  float* gk;              // [BH][Nb][2][128] group key means
-  float* gv;              // [BH][Nb][2][128] group value means
-  int* gcount;            // [BH][Nb][2]    group sizes
+  __nv_bfloat16* gk_h;    // [BH][Nb][2][128] group key means (BF16, tail MMA operand)
+  __nv_bfloat16* gv_h;    // [BH][Nb][2][128] group value means (BF16, tail MMA operand)
+  float* glog2n;          // [BH][Gp]       log2 of the group sizes, -inf for empty groups and
+                          //                the padding up to Gp = 2 Nb rounded up to 128
   float* tail_logz;       // [BH][Na]       log Z_a (-inf for an empty tail)
   float* tail_mu;         // [BH][Na][128]
   float* tail_nu;         // [BH][Na][128]
@@ -72,6 +74,9 @@ void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, 
 // Sol-Attn2 prep (sol2_tail.cu)
 void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
                    const Work& w, cudaStream_t st);
-void launch_anchor_tail(const Shape& s, const Work& w, cudaStream_t st);
+// Sol-Attn2 tail statistics on the tensor cores (sol2_tail_tc.cu); maps = anchor means, group key
+// means, group value means (BF16, 3-D, box 64 x 128 x 1, 128-byte swizzle).
+cudaError_t launch_tail_tc(const void* maps, const Shape& s, const Work& w, int* status, cudaStream_t st);
+__host__ __device__ inline int tail_groups_padded(const Shape& s) { return (2 * s.Nb + 127) / 128 * 128; }
 
 }  // namespace sol

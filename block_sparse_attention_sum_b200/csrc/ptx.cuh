@@ -227,6 +227,14 @@ __device__ __forceinline__ void tmem_st32_at(uint32_t taddr, const uint32_t (&r)
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// After tmem_ld_wait(): marks the destination registers of the preceding tcgen05.ld as (re)defined
+// here, so the compiler cannot schedule a use of them before the wait (no instruction is emitted).
+template <int kN>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[kN]) {
+#pragma unroll
+  for (int i = 0; i < kN; ++i) asm volatile("" : "+r"(r[i]));
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -107,8 +107,14 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
       w.vbar_h[o] = __float2bfloat16_rn(sv / fn);
       if (anchors) {
         const size_t a0 = (bh * s.Na + 2 * (size_t)j) * kHeadDim + c;
-        w.qanchor[a0] = sqlo / (float)nlo;
-        if (nhi > 0) w.qanchor[a0 + kHeadDim] = sqhi / (float)nhi;
+        const float alo = sqlo / (float)nlo;
+        w.qanchor[a0] = alo;
+        w.qanchor_h[a0] = __float2bfloat16_rn(alo);
+        if (nhi > 0) {
+          const float ahi = sqhi / (float)nhi;
+          w.qanchor[a0 + kHeadDim] = ahi;
+          w.qanchor_h[a0 + kHeadDim] = __float2bfloat16_rn(ahi);
+        }
       }
     }
   }
