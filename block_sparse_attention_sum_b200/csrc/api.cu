@@ -107,6 +107,9 @@ size_t carve(const Shape& s, bool sol2, char* base, Work* w) {
   t.kbar = reinterpret_cast<float*>(take(bh * nb * d * 4));
   t.kbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
   t.vbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.qbar_hi = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.qbar_lo = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.kbar_lo = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
   t.kcov = reinterpret_cast<float*>(take(bh * d * d * 4));
   t.gram_partial = reinterpret_cast<float*>(take(bh * 8 * d * d * 4));
   t.kmean = reinterpret_cast<double*>(take(bh * d * 8));
@@ -235,7 +238,13 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   launch_summary(q, k, v, s, ww, anchors, st);
   launch_kstats(s, ww, st);
   launch_thresh(s, ww, tau, diag, st);
-  launch_route(s, ww, sb0, sb1, st);
+  CUtensorMap rmaps[4];
+  int rc;
+  if ((rc = encode_rows(&rmaps[0], w.qbar_hi, s.Nb, s)) || (rc = encode_rows(&rmaps[1], w.qbar_lo, s.Nb, s)) ||
+      (rc = encode_rows(&rmaps[2], w.kbar_h, s.Nb, s)) || (rc = encode_rows(&rmaps[3], w.kbar_lo, s.Nb, s)))
+    return rc;
+  cudaError_t e = launch_route_tc(rmaps, s, ww, sb0, sb1, d.status, st);
+  if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "routing launch: %s", cudaGetErrorString(e));
   *launches += 6;
   d.last_total_pairs = (long long)s.BH * s.Nb * s.Nb;
   return check_launch("routing kernels");

@@ -18,8 +18,10 @@
 //    exp(a_j) Vhat_j are exactly the surrogate's denominator and numerator terms.
 //  * Warp roles: warp 0 TMA producer (derives the tile list from the routing bitmask), warp 1 TMEM
 //    owner and S = Q K^T issuer, warp 2 O += P V issuer, warps 4-11 two softmax warpgroups (TMEM
-//    lane = row; each warpgroup owns 64 of the 128 columns of S, P and O).  S and P are
-//    double-buffered in TMEM; O accumulates in TMEM.
+//    lane = row; each warpgroup owns 64 of the 128 columns of S, P and O).  S has one buffer in
+//    TMEM, released as soon as both warpgroups have loaded it into registers, so the next tile's
+//    Q K^T runs while this tile's softmax computes; P (BF16) has its own double buffer; O
+//    accumulates in TMEM.
 //  * Online softmax in base 2 with a lazily updated reference max: O and l are rescaled only when a
 //    row's max grows by more than 2^8, which keeps every probability <= 256.
 #include <cuda.h>
@@ -38,9 +40,10 @@ constexpr int kDescRing = 8;                   // tile descriptors in flight (pr
                                                // the MMAs, MMAs <= 2 ahead of the softmax)
 constexpr uint32_t kTileBytes = 128 * 64 * 2;  // 128 rows x 64 BF16 columns (one swizzled half, 16 KB)
 constexpr uint32_t kBoxBytes = 64 * 64 * 2;    // one 64-row x 64-column BF16 TMA box (8 KB)
-// TMEM columns: S double buffer (P of each half is written over that half's S columns once they
-// are read), and one O accumulator per softmax warpgroup (each over its half of every tile's keys).
-constexpr uint32_t kColS = 0, kColO = 256;
+// TMEM columns: S (128 x 128 FP32), P double buffer (two x 64 columns, each 128 x 128 BF16 with
+// keys 2c, 2c + 1 packed in column c; warpgroup w owns columns 32 w .. 32 w + 31), and one O
+// accumulator per softmax warpgroup (each over its half of every tile's keys).
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
 
 enum : uint32_t { kTilePair = 0, kTileSingle = 1, kTilePooled = 2 };
 
@@ -57,7 +60,7 @@ struct __align__(1024) FwdSmem {
   TileDesc desc[kDescRing];
   uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
   uint64_t dfull[kDescRing];
-  uint64_t qfull, sfull[2], sfree[2], pready[2], pvdone[2], mmadone, mmadone2;
+  uint64_t qfull, sfull, sread, pready[2], pvdone[2], mmadone, mmadone2;
   uint64_t lbar;            // softmax warpgroups: (max, sum) exchange before the epilogue merge
   float xm[2][128], xl[2][128];   // [warpgroup][row] running max and row sum, for the epilogue merge
   uint32_t tmem_base;
@@ -155,9 +158,9 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int s = 0; s < kDescRing; ++s) mbar_init(&sm.dfull[s], 1);
     mbar_init(&sm.qfull, 1);
+    mbar_init(&sm.sfull, 1);
+    mbar_init(&sm.sread, 256);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.sfull[i], 1);
-      mbar_init(&sm.sfree[i], 1);
       mbar_init(&sm.pready[i], 128);
       mbar_init(&sm.pvdone[i], 1);
     }
@@ -285,9 +288,8 @@ __global__ void __launch_bounds__(384, 1)
           break;
         }
         const TileDesc d = sm.desc[t % kDescRing];
-        const int bsel = t & 1;
-        // the buffer's previous tile (t - 2): its P was read by that tile's P V
-        if (t >= 2 && !mbar_wait(&sm.sfree[bsel], ((t >> 1) - 1) & 1, abort)) {
+        // S still holds tile t - 1 until both softmax warpgroups have loaded it
+        if (t >= 1 && !mbar_wait(&sm.sread, (t - 1) & 1, abort)) {
           ok = false;
           break;
         }
@@ -297,10 +299,10 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t k_base = smem_u32(&sm.k[s][0][0]);
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kTileBytes + (kk & 3) * 32;
-          umma_ss(tmem + kColS + 128 * bsel, sdesc_sw128(q_base + off, 16, 1024),
+          umma_ss(tmem + kColS, sdesc_sw128(q_base + off, 16, 1024),
                   sdesc_sw128(k_base + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&sm.sfull[bsel]);
+        umma_commit(&sm.sfull);
         umma_commit(&sm.kempty[s]);
         if (d.flags & 0x100u) break;
       }
@@ -336,7 +338,7 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           const bool skip = (w == 1 && d.kind == kTileSingle);   // no keys in the second half
           if (!skip) {
-            const uint32_t p_col = tmem + kColS + 128 * bsel + 64 * w;   // P_w over its S columns
+            const uint32_t p_col = tmem + kColP + 64 * bsel + 32 * w;   // P_w: 64 keys in 32 columns
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = sdesc_sw128(v_base + (4 * w + kk) * 2048, kTileBytes, 1024);
               const bool acc = w == 0 ? (u > 0 || kk > 0) : (b_started || kk > 0);
@@ -347,7 +349,6 @@ __global__ void __launch_bounds__(384, 1)
           umma_commit(&sm.pvdone[w]);
         }
         if (!ok) break;
-        umma_commit(&sm.sfree[bsel]);
         umma_commit(&sm.vempty[s]);
         if (d.flags & 0x100u) break;
       }
@@ -417,7 +418,7 @@ __global__ void __launch_bounds__(384, 1)
     for (;; ++t) {
       const int bsel = t & 1;
       if (!mbar_wait(&sm.dfull[t % kDescRing], (t / kDescRing) & 1, abort) ||
-          !mbar_wait(&sm.sfull[bsel], (t >> 1) & 1, abort)) {
+          !mbar_wait(&sm.sfull, t & 1, abort)) {
         ok = false;
         break;
       }
@@ -426,7 +427,8 @@ __global__ void __launch_bounds__(384, 1)
       const bool single = d.kind == kTileSingle;
       o1_written = o1_written || !single;
       const bool pooled = d.kind == kTilePooled;
-      const uint32_t s_addr = lane_addr + kColS + 128 * bsel + 64 * wg;
+      const uint32_t s_addr = lane_addr + kColS + 64 * wg;
+      const uint32_t p_addr = lane_addr + kColP + 64 * bsel + 32 * wg;
       // columns of this warpgroup's half that are valid for its row (warp-uniform)
       int lim_own = 64;
       if (!pooled) {
@@ -440,6 +442,9 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32_at<32>(s_addr + 32, own);
         tmem_ld_wait();
       }
+      // S is in registers: the next tile's Q K^T may overwrite it
+      tc_fence_before();
+      mbar_arrive(&sm.sread);
       // x: this warpgroup's 64 columns in place over the raw scores.  Exact tiles keep raw scores
       // (the base-2 scale is folded into the exponent), pooled tiles carry scale and log2(n_j) bias.
       float* x = reinterpret_cast<float*>(own);
@@ -498,13 +503,14 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float2 rsa = unf2(add2(rs2[0], rs2[1]));
       l = l * alpha + (rsa.x + rsa.y);
-      // O_w must be quiet (P V of tile t - 1 done) before it is rescaled
+      // P V of tile t - 1 (and so of t - 2, which read this P buffer) must have completed: O_w is
+      // rescaled below and P_bsel overwritten
       if (t > 0 && !mbar_wait(&sm.pvdone[wg], (t - 1) & 1, abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (!(single && wg == 1)) tmem_st32_at<0>(s_addr, pk);   // P over this half's S columns
+      if (!(single && wg == 1)) tmem_st32(p_addr, pk);
       // tcgen05.ld / st are warp-collective: the warp rescales if any of its rows needs it
       const bool need = upd && t > 0 && m_ref != -INFINITY;
       if (__any_sync(0xffffffffu, need)) {

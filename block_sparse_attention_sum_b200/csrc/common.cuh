@@ -40,6 +40,9 @@ struct Work {
   float* kbar;            // [BH][Nb][128]  block means of K
   __nv_bfloat16* kbar_h;  // [BH][Nb][128]  BF16 copy of kbar (surrogate MMA operand)
   __nv_bfloat16* vbar_h;  // [BH][Nb][128]  BF16 block means of V (surrogate MMA operand)
+  __nv_bfloat16* qbar_hi; // [BH][Nb][128]  bf16(qbar)            } two-term BF16 splits of the
+  __nv_bfloat16* qbar_lo; // [BH][Nb][128]  bf16(qbar - qbar_hi)  } means for the routing product
+  __nv_bfloat16* kbar_lo; // [BH][Nb][128]  bf16(kbar - kbar_h)   } (kbar_h is the hi part of kbar)
   float* kcov;            // [BH][128][128] centred covariance of the key-block means
   float* gram_partial;    // [BH][8][128][128] partial Gram sums over ranges of key blocks
   double* kmean;          // [BH][128]      mean of the key-block means
@@ -68,7 +71,10 @@ void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_b
                     const Work& w, bool anchors, cudaStream_t st);
 void launch_kstats(const Shape& s, const Work& w, cudaStream_t st);
 void launch_thresh(const Shape& s, const Work& w, float tau, bool diag, cudaStream_t st);
-void launch_route(const Shape& s, const Work& w, int sink_b0, int sink_b1, cudaStream_t st);
+// Routing on the tensor cores (route_tc.cu); maps = qbar_hi, qbar_lo, kbar_h, kbar_lo (BF16, 3-D,
+// box 64 x 128 x 1, 128-byte swizzle).
+cudaError_t launch_route_tc(const void* maps, const Shape& s, const Work& w, int sink_b0, int sink_b1, int* status,
+                            cudaStream_t st);
 void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, cudaStream_t st);
 
 // Sol-Attn2 prep (sol2_tail.cu)

@@ -64,6 +64,9 @@ size_t na_carve(const Shape& s, unsigned char* base, Work* w) {
   t.kbar = reinterpret_cast<float*>(take(bh * nb * d * 4));
   t.kbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
   t.vbar_h = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.qbar_hi = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.qbar_lo = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
+  t.kbar_lo = reinterpret_cast<__nv_bfloat16*>(take(bh * nb * d * 2));
   t.kcov = reinterpret_cast<float*>(take(bh * d * d * 4));
   t.gram_partial = reinterpret_cast<float*>(take(bh * 8 * d * d * 4));
   t.kmean = reinterpret_cast<double*>(take(bh * d * 8));
@@ -155,7 +158,7 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   na_carve(s, d.scratch, &w);
   w.stats = d.stats;
 
-  CUtensorMap maps[5];
+  CUtensorMap maps[9];
   const cuuint64_t dims4[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
   const cuuint64_t str4[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)H * kHeadDim * 2, (cuuint64_t)N * H * kHeadDim * 2};
   const cuuint32_t box4[4] = {64, 1, 64, 1};
@@ -166,7 +169,11 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   if ((rc = na_encode(enc, &maps[0], q, 4, dims4, str4, box4)) || (rc = na_encode(enc, &maps[1], k, 4, dims4, str4, box4)) ||
       (rc = na_encode(enc, &maps[2], v, 4, dims4, str4, box4)) ||
       (rc = na_encode(enc, &maps[3], w.kbar_h, 3, dims3, str3, box3)) ||
-      (rc = na_encode(enc, &maps[4], w.vbar_h, 3, dims3, str3, box3)))
+      (rc = na_encode(enc, &maps[4], w.vbar_h, 3, dims3, str3, box3)) ||
+      (rc = na_encode(enc, &maps[5], w.qbar_hi, 3, dims3, str3, box3)) ||
+      (rc = na_encode(enc, &maps[6], w.qbar_lo, 3, dims3, str3, box3)) ||
+      (rc = na_encode(enc, &maps[7], w.kbar_h, 3, dims3, str3, box3)) ||
+      (rc = na_encode(enc, &maps[8], w.kbar_lo, 3, dims3, str3, box3)))
     return rc;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -193,7 +200,8 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   launch_summary(qh, kh, vh, s, w, false, st);
   launch_kstats(s, w, st);
   launch_thresh(s, w, tau, false, st);
-  launch_route(s, w, sb0, sb1, st);
+  cudaError_t re = launch_route_tc(&maps[5], s, w, sb0, sb1, d.status, st);
+  if (re != cudaSuccess) return na_fail(SOL_ERR_LAUNCH, cudaGetErrorString(re));
   FwdParams p{};
   p.N = N;
   p.H = H;

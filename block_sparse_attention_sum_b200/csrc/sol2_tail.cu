@@ -29,121 +29,116 @@ __global__ void qdir_kernel(Shape s, Work w) {
 }
 
 // Two groups per key block: group 1 = keys with k.u > Kbar_j.u, group 0 = the rest (FP32 decision).
-// Same access pattern as the block-summary kernel: one CTA per (key block, batch), heads in turn.
+// One CTA per (key block j, b, h), the block-summary kernel's access pattern: 16 threads cover a
+// 256-byte row with 16-byte loads, 16 row groups cover the block, all loads issued up front.
 __global__ void __launch_bounds__(256) groups_kernel(const __nv_bfloat16* __restrict__ k,
                                                      const __nv_bfloat16* __restrict__ v, Shape s, Work w) {
   __shared__ float red[8][4][kHeadDim];
-  __shared__ float cut_s;
   __shared__ int n1_s;
-  const int j = blockIdx.x, b = blockIdx.y;
+  const int j = blockIdx.x, bh = blockIdx.y, b = bh / s.H, h = bh % s.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c16 = tid & 15, rg = tid >> 4;
   const int t0 = j * kBlock;
   const int n = min(kBlock, s.N - t0);
-  for (int h = 0; h < s.H; ++h) {
-    const size_t bh = (size_t)b * s.H + h;
-    const float* u = w.qdir + bh * kHeadDim;
-    if (warp == 0) {
-      const float* kb = w.kbar + (bh * s.Nb + j) * kHeadDim;
-      float acc = 0.f;
-      for (int c = lane; c < kHeadDim; c += 32) acc = fmaf(kb[c], u[c], acc);
+  if (tid == 0) n1_s = 0;
+  uint4 rk[4], rv[4];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) {
-        cut_s = acc;
-        n1_s = 0;
-      }
+  for (int m = 0; m < 4; ++m) {
+    const int r = rg + 16 * m;
+    if (r < n) {
+      const size_t off = ((size_t)(b * (size_t)s.N + t0 + r) * s.H + h) * kHeadDim + 8 * c16;
+      rk[m] = __ldg(reinterpret_cast<const uint4*>(k + off));
+      rv[m] = __ldg(reinterpret_cast<const uint4*>(v + off));
+    } else {
+      rk[m] = rv[m] = make_uint4(0, 0, 0, 0);
     }
-    float uu[8];
+  }
+  // the cut Kbar_j . u, reduced over the 16 lanes of a row group (each holds 8 channels)
+  const float* u = w.qdir + (size_t)bh * kHeadDim + 8 * c16;
+  const float* kb = w.kbar + ((size_t)bh * s.Nb + j) * kHeadDim + 8 * c16;
+  float uu[8];
+  float cut = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) uu[e] = u[8 * c16 + e];
-    __syncthreads();
-    const float cut = cut_s;
-    float k0[8], k1[8], v0[8], v1[8];
+  for (int e = 0; e < 8; ++e) {
+    uu[e] = u[e];
+    cut = fmaf(kb[e], uu[e], cut);
+  }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) k0[e] = k1[e] = v0[e] = v1[e] = 0.f;
-    int n1 = 0;
+  for (int o = 8; o > 0; o >>= 1) cut += __shfl_xor_sync(0xffffffffu, cut, o);
+  float k0[8], k1[8], v0[8], v1[8];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int r = rg + 16 * m;
-      const bool valid = r < n;   // uniform across the 16 lanes of the row
-      uint4 rk = make_uint4(0, 0, 0, 0), rv = make_uint4(0, 0, 0, 0);
-      if (valid) {
-        const size_t off = ((size_t)(b * (size_t)s.N + t0 + r) * s.H + h) * kHeadDim + 8 * c16;
-        rk = __ldg(reinterpret_cast<const uint4*>(k + off));
-        rv = __ldg(reinterpret_cast<const uint4*>(v + off));
-      }
-      float fk[8], fv[8];
-      const __nv_bfloat162* pk = reinterpret_cast<const __nv_bfloat162*>(&rk);
-      const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&rv);
+  for (int e = 0; e < 8; ++e) k0[e] = k1[e] = v0[e] = v1[e] = 0.f;
+  int n1 = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 a = __bfloat1622float2(pk[e]);
-        const float2 c = __bfloat1622float2(pv[e]);
-        fk[2 * e] = a.x;
-        fk[2 * e + 1] = a.y;
-        fv[2 * e] = c.x;
-        fv[2 * e + 1] = c.y;
-      }
-      float proj = 0.f;
+  for (int m = 0; m < 4; ++m) {
+    const bool valid = rg + 16 * m < n;   // uniform across the 16 lanes of the row
+    float fk[8], fv[8];
+    const __nv_bfloat162* pk = reinterpret_cast<const __nv_bfloat162*>(&rk[m]);
+    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&rv[m]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) proj = fmaf(fk[e], uu[e], proj);
-      // the 16 lanes of one row are lanes (lane & 16) .. (lane & 16) + 15
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) proj += __shfl_xor_sync(0xffffffffu, proj, o);
-      const bool upper = valid && proj > cut;
-      if (valid && c16 == 0 && upper) ++n1;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (upper) {
-          k1[e] += fk[e];
-          v1[e] += fv[e];
-        } else {
-          k0[e] += fk[e];
-          v0[e] += fv[e];
-        }
-      }
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = __bfloat1622float2(pk[e]);
+      const float2 c = __bfloat1622float2(pv[e]);
+      fk[2 * e] = a.x;
+      fk[2 * e + 1] = a.y;
+      fv[2 * e] = c.x;
+      fv[2 * e + 1] = c.y;
     }
+    float proj = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) proj = fmaf(fk[e], uu[e], proj);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) proj += __shfl_xor_sync(0xffffffffu, proj, o);
+    const bool upper = valid && proj > cut;
+    n1 += upper ? 1 : 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      k0[e] += __shfl_xor_sync(0xffffffffu, k0[e], 16);
-      k1[e] += __shfl_xor_sync(0xffffffffu, k1[e], 16);
-      v0[e] += __shfl_xor_sync(0xffffffffu, v0[e], 16);
-      v1[e] += __shfl_xor_sync(0xffffffffu, v1[e], 16);
+      k1[e] += upper ? fk[e] : 0.f;
+      v1[e] += upper ? fv[e] : 0.f;
+      k0[e] += upper ? 0.f : fk[e];
+      v0[e] += upper ? 0.f : fv[e];
     }
-    if (c16 == 0 && n1) atomicAdd(&n1_s, n1);
-    if (lane < 16) {
+  }
+  // rows rg and rg + 1 of a warp live in lanes l and l ^ 16
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        red[warp][0][8 * c16 + e] = k0[e];
-        red[warp][1][8 * c16 + e] = k1[e];
-        red[warp][2][8 * c16 + e] = v0[e];
-        red[warp][3][8 * c16 + e] = v1[e];
-      }
-    }
-    __syncthreads();
-    if (tid < kHeadDim) {
-      const int c = tid;
-      float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+  for (int e = 0; e < 8; ++e) {
+    k0[e] += __shfl_xor_sync(0xffffffffu, k0[e], 16);
+    k1[e] += __shfl_xor_sync(0xffffffffu, k1[e], 16);
+    v0[e] += __shfl_xor_sync(0xffffffffu, v0[e], 16);
+    v1[e] += __shfl_xor_sync(0xffffffffu, v1[e], 16);
+  }
+  __syncthreads();   // n1_s initialised
+  if (c16 == 0 && n1) atomicAdd(&n1_s, n1);
+  if (lane < 16) {
 #pragma unroll
-      for (int ww = 0; ww < 8; ++ww) {
-        a0 += red[ww][0][c];
-        a1 += red[ww][1][c];
-        b0 += red[ww][2][c];
-        b1 += red[ww][3][c];
-      }
-      const int cnt1 = n1_s, cnt0 = n - cnt1;
-      const size_t g0 = ((bh * s.Nb + j) * 2) * kHeadDim + c;
-      w.gk_h[g0] = __float2bfloat16_rn(cnt0 ? a0 / (float)cnt0 : 0.f);
-      w.gv_h[g0] = __float2bfloat16_rn(cnt0 ? b0 / (float)cnt0 : 0.f);
-      w.gk_h[g0 + kHeadDim] = __float2bfloat16_rn(cnt1 ? a1 / (float)cnt1 : 0.f);
-      w.gv_h[g0 + kHeadDim] = __float2bfloat16_rn(cnt1 ? b1 / (float)cnt1 : 0.f);
-      if (c < 2) {
-        const int cnt = c == 0 ? cnt0 : cnt1;
-        w.glog2n[bh * tail_groups_padded(s) + 2 * j + c] = cnt > 0 ? log2f((float)cnt) : -INFINITY;
-      }
+    for (int e = 0; e < 8; ++e) {
+      red[warp][0][8 * c16 + e] = k0[e];
+      red[warp][1][8 * c16 + e] = k1[e];
+      red[warp][2][8 * c16 + e] = v0[e];
+      red[warp][3][8 * c16 + e] = v1[e];
     }
-    __syncthreads();
+  }
+  __syncthreads();
+  if (tid < kHeadDim) {
+    const int c = tid;
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) {
+      a0 += red[ww][0][c];
+      a1 += red[ww][1][c];
+      b0 += red[ww][2][c];
+      b1 += red[ww][3][c];
+    }
+    const int cnt1 = n1_s, cnt0 = n - cnt1;
+    const size_t g0 = (((size_t)bh * s.Nb + j) * 2) * kHeadDim + c;
+    w.gk_h[g0] = __float2bfloat16_rn(cnt0 ? a0 / (float)cnt0 : 0.f);
+    w.gv_h[g0] = __float2bfloat16_rn(cnt0 ? b0 / (float)cnt0 : 0.f);
+    w.gk_h[g0 + kHeadDim] = __float2bfloat16_rn(cnt1 ? a1 / (float)cnt1 : 0.f);
+    w.gv_h[g0 + kHeadDim] = __float2bfloat16_rn(cnt1 ? b1 / (float)cnt1 : 0.f);
+    if (c < 2) {
+      const int cnt = c == 0 ? cnt0 : cnt1;
+      w.glog2n[(size_t)bh * tail_groups_padded(s) + 2 * j + c] = cnt > 0 ? log2f((float)cnt) : -INFINITY;
+    }
   }
 }
 
@@ -151,7 +146,7 @@ void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bf
                    const Work& w, cudaStream_t st) {
   (void)q;
   qdir_kernel<<<s.BH, kHeadDim, 0, st>>>(s, w);
-  groups_kernel<<<dim3(s.Nb, s.B), 256, 0, st>>>(k, v, s, w);
+  groups_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(k, v, s, w);
 }
 
 }  // namespace sol

@@ -101,9 +101,14 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
       const size_t o = (bh * s.Nb + j) * kHeadDim + c;
       const float fn = (float)n;
       const float kb = sk / fn;
-      w.qbar[o] = (sqlo + sqhi) / fn;
+      const float qb = (sqlo + sqhi) / fn;
+      w.qbar[o] = qb;
       w.kbar[o] = kb;
-      w.kbar_h[o] = __float2bfloat16_rn(kb);
+      const __nv_bfloat16 qh = __float2bfloat16_rn(qb), kh = __float2bfloat16_rn(kb);
+      w.qbar_hi[o] = qh;
+      w.qbar_lo[o] = __float2bfloat16_rn(qb - __bfloat162float(qh));
+      w.kbar_h[o] = kh;
+      w.kbar_lo[o] = __float2bfloat16_rn(kb - __bfloat162float(kh));
       w.vbar_h[o] = __float2bfloat16_rn(sv / fn);
       if (anchors) {
         const size_t a0 = (bh * s.Na + 2 * (size_t)j) * kHeadDim + c;
@@ -272,138 +277,6 @@ __global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau,
   }
 }
 
-// -------------------------------------------------------------------------------------------------
-// Routing: bit j of row i is set iff s_ij = s * Qbar_i . Kbar_j > tau_i (FP32), |i - j| <= 1, or
-// block j overlaps the sink.  The proxies are consumed as they are produced (only the bitmask and
-// per-row counts reach memory).  Grid (ceil(Nb / 64), BH); a 64 x 64 tile of proxies per step,
-// 4 x 4 per thread from transposed shared-memory tiles.
-// -------------------------------------------------------------------------------------------------
-constexpr int kRouteRows = 64, kRouteCols = 128;
-constexpr int kRoutePadQ = kRouteRows + 4, kRoutePadK = kRouteCols + 4;
-
-__global__ void __launch_bounds__(128) route_kernel(Shape s, Work w, int sink_b0, int sink_b1) {
-  extern __shared__ __align__(16) float rsm[];
-  float* Qt = rsm;                                  // [128][68]   Qbar^T of the 64 query blocks
-  float* Kt = rsm + kHeadDim * kRoutePadQ;          // [128][132]  Kbar^T of 128 key blocks
-  __shared__ float th[kRouteRows];
-  __shared__ int cnt[kRouteRows];
-  const int bh = blockIdx.y, i0 = blockIdx.x * kRouteRows, tid = threadIdx.x, lane = tid & 31;
-  const int ti = tid >> 4, tj = tid & 15;           // rows 8 ti .. 8 ti + 7, columns 8 tj .. 8 tj + 7
-  const float* qb = w.qbar + (size_t)bh * s.Nb * kHeadDim;
-  const float* kb = w.kbar + (size_t)bh * s.Nb * kHeadDim;
-  {
-    // thread = (row, half of the channels); 16-byte loads, eight in flight; the transposed stores
-    // of a warp hit 32 consecutive rows (no bank conflicts)
-    const int row = tid & 63, c0 = (tid >> 6) * 64;
-    const bool in = i0 + row < s.Nb;
-    const float4* src = reinterpret_cast<const float4*>(qb + (size_t)(i0 + row) * kHeadDim + c0);
-#pragma unroll
-    for (int k0 = 0; k0 < 16; k0 += 8) {
-      float4 v[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (in) v[k] = __ldg(src + k0 + k);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int c = c0 + 4 * (k0 + k);
-        Qt[(c + 0) * kRoutePadQ + row] = v[k].x;
-        Qt[(c + 1) * kRoutePadQ + row] = v[k].y;
-        Qt[(c + 2) * kRoutePadQ + row] = v[k].z;
-        Qt[(c + 3) * kRoutePadQ + row] = v[k].w;
-      }
-    }
-  }
-  if (tid < kRouteRows) {
-    th[tid] = (i0 + tid < s.Nb) ? w.thresh[(size_t)bh * s.Nb + i0 + tid] : 0.f;
-    cnt[tid] = 0;
-  }
-  for (int j0 = 0; j0 < s.Nb; j0 += kRouteCols) {
-    __syncthreads();
-    {
-      // thread = key block row; 16-byte loads, eight in flight; conflict-free transposed stores
-      const int row = tid;
-      const bool in = j0 + row < s.Nb;
-      const float4* src = reinterpret_cast<const float4*>(kb + (size_t)(j0 + row) * kHeadDim);
-#pragma unroll
-      for (int k0 = 0; k0 < 32; k0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (in) v[k] = __ldg(src + k0 + k);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int c = 4 * (k0 + k);
-          Kt[(c + 0) * kRoutePadK + row] = v[k].x;
-          Kt[(c + 1) * kRoutePadK + row] = v[k].y;
-          Kt[(c + 2) * kRoutePadK + row] = v[k].z;
-          Kt[(c + 3) * kRoutePadK + row] = v[k].w;
-        }
-      }
-    }
-    __syncthreads();
-    float acc[8][8];
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
-#pragma unroll 2
-    for (int d = 0; d < kHeadDim; ++d) {
-      const float4 q0 = *reinterpret_cast<const float4*>(&Qt[d * kRoutePadQ + 8 * ti]);
-      const float4 q1 = *reinterpret_cast<const float4*>(&Qt[d * kRoutePadQ + 8 * ti + 4]);
-      const float4 k0 = *reinterpret_cast<const float4*>(&Kt[d * kRoutePadK + 8 * tj]);
-      const float4 k1 = *reinterpret_cast<const float4*>(&Kt[d * kRoutePadK + 8 * tj + 4]);
-      const float av[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      const float bv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(av[a], bv[c], acc[a][c]);
-    }
-    // 8 rows x 8 columns of decisions -> one byte per row, OR-combined across the 4 lanes that
-    // share a 32-column word (lanes differing in their two lowest bits).
-#pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const int il = 8 * ti + a;
-      const int i = i0 + il;
-      uint32_t bits = 0;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int jj = j0 + 8 * tj + c;
-        const float shat = acc[a][c] * kScale;
-        if (jj < s.Nb && shat > th[il]) bits |= 1u << (8 * (tj & 3) + c);
-      }
-      bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
-      bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
-      if ((lane & 3) == 0 && i < s.Nb) {
-        const int wd = (j0 >> 5) + (tj >> 2);
-        if (wd < s.Nw) {
-          const int jb = 32 * wd;
-          for (int jj = max(i - 1, jb); jj <= min(i + 1, jb + 31); ++jj)
-            if (jj >= 0 && jj < s.Nb) bits |= 1u << (jj - jb);
-          if (sink_b0 <= sink_b1) {
-            const int lo = max(sink_b0, jb), hi = min(sink_b1, jb + 31);
-            for (int jj = lo; jj <= hi; ++jj) bits |= 1u << (jj - jb);
-          }
-          w.mask[((size_t)bh * s.Nb + i) * s.Nw + wd] = bits;
-          atomicAdd(&cnt[il], __popc(bits));
-        }
-      }
-    }
-  }
-  __syncthreads();
-  if (tid < kRouteRows && i0 + tid < s.Nb) {
-    const int c = cnt[tid];
-    w.rowcount[(size_t)bh * s.Nb + i0 + tid] = c;
-    atomicAdd(&w.stats[0], (unsigned long long)c);
-    atomicMin(&w.stats[1], (unsigned long long)c);
-    atomicMax(&w.stats[2], (unsigned long long)c);
-  }
-}
-
 // Expand the bitmask into one byte per (query block, key block) pair (introspection only).
 __global__ void expand_mask_kernel(Shape s, Work w, unsigned char* out) {
   const size_t total = (size_t)s.BH * s.Nb * s.Nb;
@@ -432,11 +305,6 @@ void launch_thresh(const Shape& s, const Work& w, float tau, bool diag, cudaStre
   thresh_kernel<<<dim3((s.Nb + 63) / 64, s.BH), 256, smem, st>>>(s, w, tau, diag ? 1 : 0);
 }
 
-void launch_route(const Shape& s, const Work& w, int sink_b0, int sink_b1, cudaStream_t st) {
-  const int smem = kHeadDim * (kRoutePadQ + kRoutePadK) * sizeof(float);
-  cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  route_kernel<<<dim3((s.Nb + kRouteRows - 1) / kRouteRows, s.BH), 128, smem, st>>>(s, w, sink_b0, sink_b1);
-}
 
 void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, cudaStream_t st) {
   expand_mask_kernel<<<1184, 256, 0, st>>>(s, w, mask_out);
