@@ -87,6 +87,23 @@ def measured_traffic(workload_name: str):
     return entry["dram_bytes_per_launch"]
 
 
+def union_useful_fraction(mask):
+    """Share of the fused kernel's exact-tile work that is useful: a work unit pairs query blocks
+    2u and 2u + 1 and computes both rows against every key block in the union of their exact sets,
+    so useful / computed = (|E_2u| + |E_2u+1|) / (rows x |E_2u | E_2u+1|).  mask: bool [B, H, Nb, Nb]."""
+    import numpy as np
+
+    m = np.asarray(mask, dtype=bool)
+    Nb = m.shape[-1]
+    if Nb % 2:
+        m = np.concatenate([m, np.zeros(m.shape[:-2] + (1, Nb), dtype=bool)], axis=-2)
+    a, b = m[..., 0::2, :], m[..., 1::2, :]
+    rows = 1 + np.any(b, axis=-1)          # a unit without a second query block has one row
+    useful = a.sum() + b.sum()
+    computed = (rows * (a | b).sum(axis=-1)).sum()
+    return float(useful / max(computed, 1))
+
+
 def load_peaks():
     if os.path.exists(PEAKS_PATH):
         with open(PEAKS_PATH) as f:
@@ -294,6 +311,9 @@ def main():
     flops_step, exact_flops_step = effective_flops(w.B, w.N, w.H, exact, total)
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
     sp = 1.0 - exact / total
+    gmask, _ = sa.debug_route(q, k, tau, w.sink_start, w.sink_tokens)
+    union_frac = union_useful_fraction(gmask.cpu().numpy())
+    del gmask
 
     # ---- end to end through the public API with host buffers (H2D inputs, D2H output each step)
     e2e = None
@@ -340,6 +360,7 @@ def main():
                                    if w.grid else w.name,
                        "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "tau": tau,
                        "target_sparsity": w.target_sparsity, "realised_sparsity": sp,
+                       "union_tile_useful_fraction": union_frac,
                        "parallelism": f"independent replicas x{world} (head/batch sharding, no exchange)",
                        "l2": "inputs 1.6 GB per rank > 126 MB L2; no flush"},
             "frac_of_peak": value / world / peak_burst, "frac_of_sustained_peak": value / world / peak_sust,

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -175,18 +176,17 @@ int validate(const void* q, const void* k, const void* v, const void* out, bool 
   return SOL_OK;
 }
 
-// Key blocks overlapping the sink range, as an inclusive block interval (b0 > b1: no sink).
-void sink_blocks(int N, int sink_start, int sink_tokens, int* b0, int* b1) {
-  *b0 = 1;
-  *b1 = 0;
+// Adds the key blocks overlapping a sink token range as an inclusive block interval.
+void add_sink(int N, int sink_start, int sink_tokens, SinkSet* set) {
   if (sink_tokens <= 0) return;
   long long start = sink_start >= 0 ? sink_start : (long long)N - sink_tokens;
   long long end = start + sink_tokens;
   if (start < 0) start = 0;
   if (end > N) end = N;
   if (end <= start) return;
-  *b0 = (int)(start / kBlock);
-  *b1 = (int)((end - 1) / kBlock);
+  set->b0[set->n] = (int)(start / kBlock);
+  set->b1[set->n] = (int)((end - 1) / kBlock);
+  ++set->n;
 }
 
 int encode_bthd(CUtensorMap* m, const void* base, const Shape& s) {
@@ -224,11 +224,11 @@ int check_launch(const char* what) {
 // Routing prefix shared by all entry points: summaries, threshold statistics, thresholds, bitmask.
 int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                 const Shape& s, const Work& w, float tau, int sink_start, int sink_tokens, bool anchors,
-                bool diag, cudaStream_t st, int* launches) {
-  int sb0, sb1;
-  sink_blocks(s.N, sink_start, sink_tokens, &sb0, &sb1);
-  const unsigned long long init[3] = {0ull, ~0ull, 0ull};
-  (void)init;
+                bool diag, const sol_attn_options* opts, cudaStream_t st, int* launches) {
+  SinkSet sinks{};
+  add_sink(s.N, sink_start, sink_tokens, &sinks);
+  if (opts)
+    for (int e = 0; e < opts->n_extra_sinks; ++e) add_sink(s.N, opts->extra_sink_start[e], opts->extra_sink_tokens[e], &sinks);
   if (cudaMemsetAsync(d.stats, 0, sizeof(unsigned long long), st) != cudaSuccess ||
       cudaMemsetAsync(d.stats + 1, 0xff, sizeof(unsigned long long), st) != cudaSuccess ||
       cudaMemsetAsync(d.stats + 2, 0, sizeof(unsigned long long), st) != cudaSuccess)
@@ -243,20 +243,30 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   if ((rc = encode_rows(&rmaps[0], w.qbar_hi, s.Nb, s)) || (rc = encode_rows(&rmaps[1], w.qbar_lo, s.Nb, s)) ||
       (rc = encode_rows(&rmaps[2], w.kbar_h, s.Nb, s)) || (rc = encode_rows(&rmaps[3], w.kbar_lo, s.Nb, s)))
     return rc;
-  cudaError_t e = launch_route_tc(rmaps, s, ww, sb0, sb1, d.status, st);
+  cudaError_t e = launch_route_tc(rmaps, s, ww, sinks, d.status, st);
   if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "routing launch: %s", cudaGetErrorString(e));
   *launches += 6;
   d.last_total_pairs = (long long)s.BH * s.Nb * s.Nb;
   return check_launch("routing kernels");
 }
 
-int check_options(const sol_attn_options* o, bool* diag) {
+// Validates the options against the sequence length; sets *diag.
+int check_options(const sol_attn_options* o, int N, bool* diag) {
   *diag = false;
   if (!o) return SOL_OK;
   for (int r : o->reserved)
     if (r != 0) return fail(SOL_ERR_OPTION, "reserved option fields must be zero");
   if (o->thresh_type != SOL_THRESH_EXACT && o->thresh_type != SOL_THRESH_DIAG)
     return fail(SOL_ERR_OPTION, "unknown thresh_type %d", o->thresh_type);
+  if (o->n_extra_sinks < 0 || o->n_extra_sinks > SOL_MAX_EXTRA_SINKS)
+    return fail(SOL_ERR_OPTION, "n_extra_sinks must be in [0, %d]", SOL_MAX_EXTRA_SINKS);
+  for (int e = 0; e < SOL_MAX_EXTRA_SINKS; ++e) {
+    const bool used = e < o->n_extra_sinks;
+    if (!used && (o->extra_sink_start[e] != 0 || o->extra_sink_tokens[e] != 0))
+      return fail(SOL_ERR_OPTION, "unused extra sink slots must be zero");
+    if (used && (o->extra_sink_start[e] < 0 || o->extra_sink_start[e] >= N || o->extra_sink_tokens[e] <= 0))
+      return fail(SOL_ERR_OPTION, "extra sink %d needs 0 <= start < N and tokens > 0", e);
+  }
   *diag = o->thresh_type == SOL_THRESH_DIAG;
   return SOL_OK;
 }
@@ -266,7 +276,7 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   int rc = validate(q, k, v, out, true, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
   bool diag;
-  if ((rc = check_options(opts, &diag))) return rc;
+  if ((rc = check_options(opts, N, &diag))) return rc;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;
   int dev;
@@ -290,7 +300,7 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   const auto* qh = static_cast<const __nv_bfloat16*>(q);
   const auto* kh = static_cast<const __nv_bfloat16*>(k);
   const auto* vh = static_cast<const __nv_bfloat16*>(v);
-  if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, diag, st, &launches))) return rc;
+  if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, diag, opts, st, &launches))) return rc;
   if (sol2) {
     CUtensorMap tmaps[3];
     if ((rc = encode_rows(&tmaps[0], w.qanchor_h, s.Na, s)) || (rc = encode_rows(&tmaps[1], w.gk_h, 2 * s.Nb, s)) ||
@@ -310,7 +320,10 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   p.Na = s.Na;
   p.QT = s.QT;
   p.mask = w.mask;
-  p.order = nullptr;
+  p.qt_begin = 0;
+  p.qt_count = s.QT;
+  p.row_lo = 0;
+  p.row_hi = N;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = d->status;
   p.qanchor = w.qanchor;
@@ -337,6 +350,62 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   return SOL_OK;
 }
 
+// Exact (dense) attention for the query tokens [q_start, q_start + q_tokens): the fused kernel
+// over the query tiles that cover them, every key block marked exact for those query blocks, and
+// only rows inside the range written.
+int dense_rows(const void* q, const void* k, const void* v, void* out, int B, int N, int H, int q_start, int q_tokens,
+               void* stream) {
+  int rc = validate(q, k, v, out, true, B, N, H, 1.0f, -1, 0);
+  if (rc) return rc;
+  if (q_tokens > 0 && q_start >= N) return fail(SOL_ERR_SINK, "q_start (%d) must be < N (%d)", q_start, N);
+  long long r0 = q_start >= 0 ? q_start : (long long)N - q_tokens;
+  long long r1 = r0 + (q_tokens > 0 ? q_tokens : 0);
+  if (r0 < 0) r0 = 0;
+  if (r1 > N) r1 = N;
+  if (r1 <= r0) return SOL_OK;   // no rows: nothing to do
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* d;
+  int dev;
+  if ((rc = device_state(&d, &dev))) return rc;
+  if ((rc = get_encode())) return rc;
+  const Shape s = make_shape(B, N, H);
+  Work w;
+  if ((rc = ensure_workspace(*d, carve(s, false, nullptr, nullptr)))) return rc;
+  carve(s, false, static_cast<char*>(d->ws), &w);
+  w.stats = d->stats;
+  // the kernel's pooled-tile maps must be valid descriptors; no pooled tile is loaded here
+  CUtensorMap maps[5];
+  if ((rc = encode_bthd(&maps[0], q, s)) || (rc = encode_bthd(&maps[1], k, s)) || (rc = encode_bthd(&maps[2], v, s)) ||
+      (rc = encode_pooled(&maps[3], w.kbar_h, s)) || (rc = encode_pooled(&maps[4], w.vbar_h, s)))
+    return rc;
+  const int qt0 = (int)(r0 / kBlock) / 2, qt1 = (int)((r1 - 1) / kBlock) / 2;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamWaitEvent(st, d->done, 0) != cudaSuccess) return fail(SOL_ERR_LAUNCH, "cudaStreamWaitEvent failed");
+  launch_dense_mask(s, w, 2 * qt0, std::min(2 * qt1 + 1, s.Nb - 1), st);
+  FwdParams p{};
+  p.N = N;
+  p.H = H;
+  p.Nb = s.Nb;
+  p.Nw = s.Nw;
+  p.Na = s.Na;
+  p.QT = s.QT;
+  p.mask = w.mask;
+  p.qt_begin = qt0;
+  p.qt_count = qt1 - qt0 + 1;
+  p.row_lo = (int)r0;
+  p.row_hi = (int)r1;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = d->status;
+  cudaError_t e = launch_attn_fwd(maps, p, s.BH * p.qt_count, false, st);
+  if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "fused attention launch: %s", cudaGetErrorString(e));
+  if ((rc = check_launch("dense rows"))) return rc;
+  cudaEventRecord(d->done, st);
+  d->last_stream = st;
+  d->last_launches = 2;
+  g_last_device = dev;
+  return SOL_OK;
+}
+
 }  // namespace
 
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
@@ -346,6 +415,7 @@ void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg)
 using namespace sol;
 
 extern "C" {
+
 
 int sol_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
                  int sink_start, int sink_tokens, void* stream) {
@@ -397,7 +467,7 @@ int sol_attn_debug_route_ex(const void* q, const void* k, int B, int N, int H, f
   int rc = validate(q, k, nullptr, nullptr, false, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
   bool diag;
-  if ((rc = check_options(opts, &diag))) return rc;
+  if ((rc = check_options(opts, N, &diag))) return rc;
   if (!mask) return fail(SOL_ERR_NULL, "mask must be non-NULL");
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;
@@ -413,8 +483,8 @@ int sol_attn_debug_route_ex(const void* q, const void* k, int B, int N, int H, f
   int launches = 0;
   // the summary kernel reads v as well; pass k, whose summaries are simply discarded
   if ((rc = run_routing(*d, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                        static_cast<const __nv_bfloat16*>(k), s, w, tau, sink_start, sink_tokens, false, diag, st,
-                        &launches)))
+                        static_cast<const __nv_bfloat16*>(k), s, w, tau, sink_start, sink_tokens, false, diag, opts,
+                        st, &launches)))
     return rc;
   launch_expand_mask(s, w, mask, st);
   if (thresh) cudaMemcpyAsync(thresh, w.thresh, (size_t)s.BH * s.Nb * sizeof(float), cudaMemcpyDeviceToDevice, st);
@@ -502,6 +572,12 @@ void sol_attn_release_workspace(void) {
     d.ws_bytes = 0;
   }
   if (cur >= 0) cudaSetDevice(cur);
+}
+
+int sol_attn_dense_rows(const void* q, const void* k, const void* v, void* out, int B, int N, int H, int q_start,
+                        int q_tokens, void* stream) {
+  g_err[0] = 0;
+  return dense_rows(q, k, v, out, B, N, H, q_start, q_tokens, stream);
 }
 
 }  // extern "C"

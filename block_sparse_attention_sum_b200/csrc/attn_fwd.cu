@@ -106,25 +106,6 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   return r;
 }
 
-// 2^y for a pair on the FMA pipe, to take load off the MUFU unit (16 results / clk / SM).
-// Range reduction y = n + f with n = round(y) (via the 1.5 * 2^23 rounding constant), f in
-// [-1/2, 1/2]; 2^f by a cubic fitted to minimise the relative error on [-1/2, 1/2] (Lawson's
-// iteration, max relative error 1.0e-4, below BF16's 2^-9); 2^n by adding n to the exponent field.
-// Inputs below -127 (and -inf) are clamped, giving 0.
-__device__ __forceinline__ float2 exp2_poly_pair(float y0, float y1) {
-  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-  const uint64_t yy = f2(fmaxf(y0, -127.f), fmaxf(y1, -127.f));
-  const uint64_t t = add2(yy, f2(kRound, kRound));
-  const uint64_t n = add2(t, f2(-kRound, -kRound));
-  const uint64_t fr = fma2(n, f2(-1.f, -1.f), yy);
-  uint64_t p = fma2(f2(0.05500893294811249f, 0.05500893294811249f), fr, f2(0.2422109693288803f, 0.2422109693288803f));
-  p = fma2(p, fr, f2(0.6932829022407532f, 0.6932829022407532f));
-  p = fma2(p, fr, f2(1.f, 1.f));
-  const float2 pf = unf2(p), tf = unf2(t);
-  return make_float2(__int_as_float(__float_as_int(pf.x) + (__float_as_int(tf.x) << 23)),
-                     __int_as_float(__float_as_int(pf.y) + (__float_as_int(tf.y) << 23)));
-}
-
 __device__ __forceinline__ void set_timeout(int* status) { atomicExch(status, kDevTimeout); }
 
 }  // namespace
@@ -143,8 +124,8 @@ __global__ void __launch_bounds__(384, 1)
   FwdSmem& sm = *reinterpret_cast<FwdSmem*>(smem_raw);
   volatile int* abort = &sm.abort;
 
-  const int unit = p.order ? p.order[blockIdx.x] : (int)blockIdx.x;
-  const int bh = unit / p.QT, qt = unit % p.QT;
+  const int unit = (int)blockIdx.x;
+  const int bh = unit / p.qt_count, qt = p.qt_begin + unit % p.qt_count;
   const int b = bh / p.H, h = bh % p.H;
   const int qb0 = 2 * qt;
   const bool has_hi = qb0 + 1 < p.Nb;
@@ -404,7 +385,7 @@ __global__ void __launch_bounds__(384, 1)
     const int hf = r >> 6;
     const int qi = qb0 + hf;
     const int tok = 64 * qb0 + r;
-    const bool row_valid = tok < p.N;
+    const bool row_valid = tok >= p.row_lo && tok < p.row_hi;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t o_addr = lane_addr + kColO + 128 * wg;
     const uint32_t* mrow = p.mask + ((size_t)bh * p.Nb + min(qi, p.Nb - 1)) * p.Nw;
@@ -487,13 +468,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float2 y = unf2(fma2(f2(x[2 * c], x[2 * c + 1]), fs2, nm2));
-          float2 pp;
-          if ((c & 3) == 3) {
-            pp = exp2_poly_pair(y.x, y.y);
-          } else {
-            pp.x = ex2(y.x);
-            pp.y = ex2(y.y);
-          }
+          const float2 pp = make_float2(ex2(y.x), ex2(y.y));
           rs2[c & 1] = add2(rs2[c & 1], f2(pp.x, pp.y));
           pk[c] = pack_bf16x2(pp.x, pp.y);
         }

@@ -10,7 +10,8 @@ namespace sol {
 struct FwdParams {
   int N, H, Nb, Nw, Na, QT;
   const uint32_t* mask;      // [BH][Nb][Nw]
-  const int* order;          // unit order (nullptr: identity)
+  int qt_begin, qt_count;    // query tiles (pairs of query blocks) qt_begin .. + qt_count - 1 of each (b, h)
+  int row_lo, row_hi;        // token rows [row_lo, row_hi) are written; the others are computed only
   __nv_bfloat16* out;        // [B][N][H][128]
   int* status;               // device status word
   // Sol-Attn2 tail (unused by Sol-Attn)

@@ -73,9 +73,17 @@ void launch_kstats(const Shape& s, const Work& w, cudaStream_t st);
 void launch_thresh(const Shape& s, const Work& w, float tau, bool diag, cudaStream_t st);
 // Routing on the tensor cores (route_tc.cu); maps = qbar_hi, qbar_lo, kbar_h, kbar_lo (BF16, 3-D,
 // box 64 x 128 x 1, 128-byte swizzle).
-cudaError_t launch_route_tc(const void* maps, const Shape& s, const Work& w, int sink_b0, int sink_b1, int* status,
+// Exact key-block ranges forced by the sinks: inclusive block intervals [b0[e], b1[e]].
+constexpr int kMaxSinkRanges = 5;   // the sink_start / sink_tokens range and up to 4 extra ranges
+struct SinkSet {
+  int n;
+  int b0[kMaxSinkRanges], b1[kMaxSinkRanges];
+};
+cudaError_t launch_route_tc(const void* maps, const Shape& s, const Work& w, const SinkSet& sinks, int* status,
                             cudaStream_t st);
 void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, cudaStream_t st);
+// Sets every valid bit of the bitmask rows of query blocks qb_lo .. qb_hi (all heads).
+void launch_dense_mask(const Shape& s, const Work& w, int qb_lo, int qb_hi, cudaStream_t st);
 
 // Sol-Attn2 prep (sol2_tail.cu)
 void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,

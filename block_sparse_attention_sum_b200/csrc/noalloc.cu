@@ -183,15 +183,16 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
       cudaMemsetAsync(d.stats + 2, 0, sizeof(unsigned long long), st) != cudaSuccess)
     return na_fail(SOL_ERR_LAUNCH, "statistics reset failed");
 
-  int sb0 = 1, sb1 = 0;
+  SinkSet sinks{};
   if (sink_tokens > 0) {
     long long start = sink_start >= 0 ? sink_start : (long long)N - sink_tokens;
     long long end = start + sink_tokens;
     if (start < 0) start = 0;
     if (end > N) end = N;
     if (end > start) {
-      sb0 = (int)(start / kBlock);
-      sb1 = (int)((end - 1) / kBlock);
+      sinks.b0[0] = (int)(start / kBlock);
+      sinks.b1[0] = (int)((end - 1) / kBlock);
+      sinks.n = 1;
     }
   }
   const auto* qh = static_cast<const __nv_bfloat16*>(q);
@@ -200,7 +201,7 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   launch_summary(qh, kh, vh, s, w, false, st);
   launch_kstats(s, w, st);
   launch_thresh(s, w, tau, false, st);
-  cudaError_t re = launch_route_tc(&maps[5], s, w, sb0, sb1, d.status, st);
+  cudaError_t re = launch_route_tc(&maps[5], s, w, sinks, d.status, st);
   if (re != cudaSuccess) return na_fail(SOL_ERR_LAUNCH, cudaGetErrorString(re));
   FwdParams p{};
   p.N = N;
@@ -210,7 +211,10 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   p.Na = s.Na;
   p.QT = s.QT;
   p.mask = w.mask;
-  p.order = nullptr;
+  p.qt_begin = 0;
+  p.qt_count = s.QT;
+  p.row_lo = 0;
+  p.row_hi = N;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = d.status;
   cudaError_t e = launch_attn_fwd(maps, p, s.BH * s.QT, false, st);

@@ -40,7 +40,7 @@ struct __align__(1024) RouteSmem {
 __global__ void __launch_bounds__(192, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tm_qhi, const __grid_constant__ CUtensorMap tm_qlo,
                     const __grid_constant__ CUtensorMap tm_khi, const __grid_constant__ CUtensorMap tm_klo,
-                    const Shape s, const Work w, int sink_b0, int sink_b1, int* status) {
+                    const Shape s, const Work w, const SinkSet sinks, int* status) {
   extern __shared__ __align__(1024) uint8_t rsm_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (smem_u32(rsm_raw) & 1023u) {
@@ -175,8 +175,8 @@ __global__ void __launch_bounds__(192, 1)
         const int jb = 128 * c + 32 * g;   // first key block of this word
         // forced blocks: adjacency and the sink; nothing beyond the last block
         for (int j = max(i - 1, jb); j <= min(i + 1, jb + 31); ++j) bits |= 1u << (j - jb);
-        if (sink_b0 <= sink_b1) {
-          const int lo = max(sink_b0, jb), hi = min(sink_b1, jb + 31);
+        for (int e = 0; e < sinks.n; ++e) {
+          const int lo = max(sinks.b0[e], jb), hi = min(sinks.b1[e], jb + 31);
           for (int j = lo; j <= hi; ++j) bits |= 1u << (j - jb);
         }
         const int nvalid = s.Nb - jb;
@@ -210,14 +210,14 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-cudaError_t launch_route_tc(const void* map_ptr, const Shape& s, const Work& w, int sink_b0, int sink_b1, int* status,
+cudaError_t launch_route_tc(const void* map_ptr, const Shape& s, const Work& w, const SinkSet& sinks, int* status,
                             cudaStream_t st) {
   const CUtensorMap* maps = static_cast<const CUtensorMap*>(map_ptr);
   const int smem = (int)sizeof(RouteSmem);
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  route_tc_kernel<<<dim3((s.Nb + 127) / 128, s.BH), 192, smem, st>>>(maps[0], maps[1], maps[2], maps[3], s, w, sink_b0,
-                                                                      sink_b1, status);
+  route_tc_kernel<<<dim3((s.Nb + 127) / 128, s.BH), 192, smem, st>>>(maps[0], maps[1], maps[2], maps[3], s, w, sinks,
+                                                                      status);
   return cudaGetLastError();
 }
 

@@ -288,6 +288,20 @@ __global__ void expand_mask_kernel(Shape s, Work w, unsigned char* out) {
   }
 }
 
+// Dense query rows: every key block exact for query blocks qb_lo + blockIdx.x.
+__global__ void dense_mask_kernel(Shape s, Work w, int qb_lo) {
+  const int i = qb_lo + blockIdx.x, bh = blockIdx.y;
+  uint32_t* row = w.mask + ((size_t)bh * s.Nb + i) * s.Nw;
+  for (int wd = threadIdx.x; wd < s.Nw; wd += blockDim.x) {
+    const int nvalid = s.Nb - 32 * wd;
+    row[wd] = nvalid >= 32 ? 0xffffffffu : ((1u << nvalid) - 1u);
+  }
+}
+
+void launch_dense_mask(const Shape& s, const Work& w, int qb_lo, int qb_hi, cudaStream_t st) {
+  dense_mask_kernel<<<dim3(qb_hi - qb_lo + 1, s.BH), 32, 0, st>>>(s, w, qb_lo);
+}
+
 void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
                     const Work& w, bool anchors, cudaStream_t st) {
   summary_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, k, v, s, w, anchors ? 1 : 0);

@@ -33,6 +33,7 @@ EXPORTS = [
     "sol_attn_last_launch_count",
     "sol_attn_release_workspace",
     "sol_attn_fwd_noalloc",
+    "sol_attn_dense_rows",
 ]
 
 STATUS = {
@@ -42,18 +43,31 @@ STATUS = {
 }
 
 THRESH_TYPES = {"exact": 0, "diag": 1}
+MAX_EXTRA_SINKS = 4
 
 
 class Options(ctypes.Structure):
     """sol_attn_options (include/sol_attn.h)."""
 
-    _fields_ = [("thresh_type", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+    _fields_ = [("thresh_type", ctypes.c_int), ("n_extra_sinks", ctypes.c_int),
+                ("extra_sink_start", ctypes.c_int * MAX_EXTRA_SINKS), ("extra_sink_tokens", ctypes.c_int * MAX_EXTRA_SINKS),
+                ("reserved", ctypes.c_int * 6)]
 
 
-def _options(thresh_type: str):
+def _options(thresh_type: str, extra_sinks=()):
+    """extra_sinks: up to MAX_EXTRA_SINKS (start, tokens) token ranges made exact for every query."""
     if thresh_type not in THRESH_TYPES:
         raise ValueError(f"thresh_type must be one of {sorted(THRESH_TYPES)}")
-    return Options(THRESH_TYPES[thresh_type])
+    extra_sinks = list(extra_sinks)
+    if len(extra_sinks) > MAX_EXTRA_SINKS:
+        raise ValueError(f"at most {MAX_EXTRA_SINKS} extra sink ranges")
+    o = Options()
+    o.thresh_type = THRESH_TYPES[thresh_type]
+    o.n_extra_sinks = len(extra_sinks)
+    for e, (start, tokens) in enumerate(extra_sinks):
+        o.extra_sink_start[e] = int(start)
+        o.extra_sink_tokens[e] = int(tokens)
+    return o
 
 
 class SolAttnError(RuntimeError):
@@ -110,6 +124,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_release_workspace.restype = None
     lib.sol_attn_fwd_noalloc.argtypes = fwd_args
     lib.sol_attn_fwd_noalloc.restype = i
+    lib.sol_attn_dense_rows.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.sol_attn_dense_rows.restype = i
     _lib = lib
     return lib
 
@@ -138,7 +154,7 @@ def _check_qkv(q, k, v=None):
     return q.shape[0], q.shape[1], q.shape[2]
 
 
-def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type="exact"):
+def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type="exact", extra_sinks=()):
     B, N, H = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
@@ -148,8 +164,8 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
     args = [q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, float(tau), int(sink_start),
             int(sink_tokens)]
     with torch.cuda.device(q.device):
-        if thresh_type != "exact":
-            opts = _options(thresh_type)
+        if thresh_type != "exact" or extra_sinks:
+            opts = _options(thresh_type, extra_sinks)
             rc = getattr(lib, fn_name + "_ex")(*args, ctypes.byref(opts), _stream_handle(stream))
         else:
             rc = getattr(lib, fn_name)(*args, _stream_handle(stream))
@@ -157,14 +173,30 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
     return out
 
 
-def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact"):
+def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
+                 extra_sinks=()):
     """Sol-Attn forward through the C ABI; returns ``out`` (BF16 [B, N, H, 128])."""
-    return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type)
+    return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks)
 
 
-def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact"):
+def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
+                  extra_sinks=()):
     """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
-    return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type)
+    return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks)
+
+
+def sol_attn_dense_rows(q, k, v, out, q_start, q_tokens, stream=None):
+    """Exact dense attention for query tokens [q_start, q_start + q_tokens) written into ``out``
+    (the other rows are left as they are); ``q_start < 0`` selects the suffix."""
+    B, N, H = _check_qkv(q, k, v)
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device != q.device:
+        raise ValueError("out must be a contiguous BF16 tensor shaped like q")
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.sol_attn_dense_rows(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, int(q_start),
+                                     int(q_tokens), _stream_handle(stream))
+    _check(rc)
+    return out
 
 
 def sol_attn_fwd_noalloc(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None):
@@ -183,7 +215,7 @@ def sol_attn2(q, k, v, tau=1.0, sink_start=None, sink_tokens=0, out=None):
     return sol_attn2_fwd(q, k, v, tau, -1 if sink_start is None else sink_start, sink_tokens, out)
 
 
-def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None, thresh_type="exact"):
+def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None, thresh_type="exact", extra_sinks=()):
     """Exact-block mask (uint8 [B, H, Nb, Nb]) and thresholds (float32 [B, H, Nb]) from the GPU router."""
     B, N, H = _check_qkv(q, k)
     Nb = math.ceil(N / BLOCK)
@@ -191,7 +223,7 @@ def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None, thresh
     thresh = torch.empty(B, H, Nb, dtype=torch.float32, device=q.device)
     lib = load_library()
     with torch.cuda.device(q.device):
-        opts = _options(thresh_type)
+        opts = _options(thresh_type, extra_sinks)
         rc = lib.sol_attn_debug_route_ex(q.data_ptr(), k.data_ptr(), B, N, H, float(tau), int(sink_start),
                                          int(sink_tokens), ctypes.byref(opts), mask.data_ptr(), thresh.data_ptr(),
                                          _stream_handle(stream))

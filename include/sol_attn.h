@@ -62,10 +62,25 @@ typedef enum {
   SOL_THRESH_DIAG = 1   /* sigma_i^2 = (Qbar_i * Qbar_i) . v_K with v_K the per-channel variance of Kbar */
 } sol_thresh_type;
 
-/* Options of the _ex entry points.  A NULL pointer means all defaults; reserved fields must be 0. */
+#define SOL_MAX_EXTRA_SINKS 4
+
+/*
+ * Options of the _ex entry points.  A NULL pointer means all defaults (an all-zero struct is the
+ * default too); reserved fields must be 0.
+ *   thresh_type        sol_thresh_type.
+ *   n_extra_sinks      0 .. SOL_MAX_EXTRA_SINKS further exact key ranges, in addition to the
+ *                      sink_start / sink_tokens range (for inputs with several text segments, e.g.
+ *                      joint attention over interleaved text and video tokens).  Range e covers
+ *                      tokens [extra_sink_start[e], extra_sink_start[e] + extra_sink_tokens[e]),
+ *                      clipped to N; it needs 0 <= start < N and tokens > 0.  Like the main sink,
+ *                      every key block overlapping a range is exact for every query.
+ */
 typedef struct {
-  int thresh_type;   /* sol_thresh_type */
-  int reserved[7];
+  int thresh_type;
+  int n_extra_sinks;
+  int extra_sink_start[SOL_MAX_EXTRA_SINKS];
+  int extra_sink_tokens[SOL_MAX_EXTRA_SINKS];
+  int reserved[6];
 } sol_attn_options;
 
 /*
@@ -97,8 +112,9 @@ int sol_attn2_fwd(const void* q, const void* k, const void* v, void* out, int B,
 /*
  * sol_attn_fwd / sol_attn2_fwd / sol_attn_debug_route with options (`opts` may be NULL).  With
  * SOL_THRESH_DIAG the threshold's variance keeps only the diagonal of the key-block-mean covariance
- * (the mean mu_i stays exact); everything else is as in the plain entry points.  An invalid option
- * returns SOL_ERR_OPTION before anything is launched.
+ * (the mean mu_i stays exact); extra sink ranges add exact key blocks as described at
+ * sol_attn_options; everything else is as in the plain entry points.  An invalid option returns
+ * SOL_ERR_OPTION before anything is launched.
  */
 int sol_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
                     int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream);
@@ -161,7 +177,7 @@ void sol_attn_release_workspace(void);
  *   - Its scratch is a fixed 64 MiB region declared at file scope in the library (plus two small
  *     status / statistics words); every GPU that loads the library holds it until the process
  *     exits.  The call never calls cudaMalloc / cudaFree or any allocating routine.  A shape whose
- *     scratch exceeds 64 MiB (for example B*H = 32 at N > ~40K tokens) returns SOL_ERR_SHAPE with a
+ *     scratch exceeds 64 MiB (for example B*H = 32 at N > ~38K tokens) returns SOL_ERR_SHAPE with a
  *     message; use sol_attn_fwd for those.
  *   - The first call on a device (with that device current) looks up the scratch region's device
  *     address; make that first call before any stream capture on the device.
@@ -173,6 +189,22 @@ void sol_attn_release_workspace(void);
  */
 int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
                          int sink_start, int sink_tokens, void* stream);
+
+/*
+ * Dense companion call for text query rows in joint (MMDiT) attention.  The Sol-Attn README,
+ * "Exact KV sink": a sink keeps the text KEY blocks exact for every query but does not make the
+ * text QUERY rows dense; an integration should use dense attention for the valid text queries and
+ * Sol-Attn for the image/video queries.  This entry point computes exact softmax attention of the
+ * query tokens [q_start, q_start + q_tokens) (clipped to N) over all N keys,
+ * o_r = sum_t exp(q_r.k_t / sqrt(128)) v_t / sum_t exp(q_r.k_t / sqrt(128)), rounded to BF16, and
+ * writes only those rows of `out`; every other row of `out` is left as it was.  Call it after
+ * sol_attn_fwd / sol_attn2_fwd on the same `out` to give the text rows dense attention.
+ *   - q_start < 0 means the suffix [N - q_tokens, N); q_tokens <= 0 is a no-op (SOL_OK).
+ *   - q_start >= N (with q_tokens > 0) returns SOL_ERR_SINK; the other argument rules are those
+ *     of sol_attn_fwd (tau and the sink do not apply).
+ */
+int sol_attn_dense_rows(const void* q, const void* k, const void* v, void* out, int B, int N, int H, int q_start,
+                        int q_tokens, void* stream);
 
 #ifdef __cplusplus
 }

@@ -54,6 +54,12 @@ R11 Sol-Attn2 anchors: anchor a covers tokens [32a, 32a + 32) (clipped to N), q_
 R12 Sol-Attn2 does not add the Sol-Attn surrogate: the complementary tail replaces it.
 R13 Routing decisions are taken on FP32-rounded proxy and threshold values (the precision the
     kernel decides in); the values themselves are computed in FP64.
+R16 Several sink ranges (the README describes one contiguous range; texts split into segments need
+    several): each range is applied as the README's sink, and a key block is exact if it overlaps
+    any of them.
+R17 Dense text rows ([README] "Exact KV sink": the sink does not make text query rows dense; an
+    MMDiT integration should use dense attention for the valid text queries): plain softmax
+    attention of those query tokens over all keys, o_r = sum_t e^{s q_r.k_t} v_t / sum_t e^{s q_r.k_t}.
 """
 from __future__ import annotations
 
@@ -158,19 +164,22 @@ def threshold_diag(Qbar: np.ndarray, Kbar: np.ndarray, tau: float):
     return mu, sigma, mu + tau * sigma
 
 
-def sink_block_flags(N: int, sink_start: int, sink_tokens: int) -> np.ndarray:
-    """Key blocks that overlap the exact sink range (README "Exact KV sink"; reading R8)."""
+def sink_block_flags(N: int, sink_start: int, sink_tokens: int, extra_sinks=()) -> np.ndarray:
+    """Key blocks that overlap an exact sink range (README "Exact KV sink"; readings R8, R16).
+
+    ``extra_sinks``: further (start, tokens) ranges with start >= 0, each applied like the first."""
     Nb = num_blocks(N)
     flags = np.zeros(Nb, dtype=bool)
-    if sink_tokens <= 0:
-        return flags
-    start = sink_start if sink_start >= 0 else N - sink_tokens
-    end = min(N, start + sink_tokens)
-    start = max(0, start)
-    for j in range(Nb):
-        a, b = block_range(j, N)
-        if a < end and b > start:
-            flags[j] = True
+    for rs, rt in [(sink_start, sink_tokens)] + list(extra_sinks):
+        if rt <= 0:
+            continue
+        start = rs if rs >= 0 else N - rt
+        end = min(N, start + rt)
+        start = max(0, start)
+        for j in range(Nb):
+            a, b = block_range(j, N)
+            if a < end and b > start:
+                flags[j] = True
     return flags
 
 
@@ -235,10 +244,11 @@ def _routing_for_head(q_bh, k_bh, tau, sink_flags, thresh_type="exact"):
                 counts=block_counts(N))
 
 
-def routing(q, k, tau: float, sink_start: int = -1, sink_tokens: int = 0, thresh_type: str = "exact"):
+def routing(q, k, tau: float, sink_start: int = -1, sink_tokens: int = 0, thresh_type: str = "exact",
+            extra_sinks=()):
     """Per (b, h): proxies, mu, sigma, thresholds and exact masks. Returns a dict of stacked arrays."""
     B, N, H, _ = q.shape
-    sink = sink_block_flags(N, sink_start, sink_tokens)
+    sink = sink_block_flags(N, sink_start, sink_tokens, extra_sinks)
     per = [[_routing_for_head(head_slice(q, b, h), head_slice(k, b, h), tau, sink, thresh_type) for h in range(H)]
            for b in range(B)]
     keys = ["shat", "mu", "sigma", "thresh", "mask"]
@@ -251,7 +261,7 @@ def _row_subset(N, qblocks):
 
 
 def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None,
-             thresh_type: str = "exact"):
+             thresh_type: str = "exact", extra_sinks=()):
     """Sol-Attn forward. Returns dict with ``out`` (FP64 [B, N, H, 128]; NaN for rows not computed),
     ``mask`` [B, H, Nb, Nb], ``shat``, ``thresh``.
 
@@ -260,7 +270,7 @@ def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qb
     """
     B, N, H, _ = q.shape
     Nb = num_blocks(N)
-    sink = sink_block_flags(N, sink_start, sink_tokens)
+    sink = sink_block_flags(N, sink_start, sink_tokens, extra_sinks)
     out = np.full((B, N, H, HEAD_DIM), np.nan)
     masks = np.zeros((B, H, Nb, Nb), dtype=bool)
     shats = np.zeros((B, H, Nb, Nb))
@@ -345,11 +355,12 @@ def sol_attn2_rows(q_rows, row0, k_bh, v_bh, mask_row, counts, kg, vg, qbar_anch
     return out
 
 
-def sol_attn2(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None):
+def sol_attn2(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None,
+              extra_sinks=()):
     """Sol-Attn2 forward (complementary tail). Same return convention as :func:`sol_attn`."""
     B, N, H, _ = q.shape
     Nb = num_blocks(N)
-    sink = sink_block_flags(N, sink_start, sink_tokens)
+    sink = sink_block_flags(N, sink_start, sink_tokens, extra_sinks)
     out = np.full((B, N, H, HEAD_DIM), np.nan)
     masks = np.zeros((B, H, Nb, Nb), dtype=bool)
     pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
@@ -365,6 +376,26 @@ def sol_attn2(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, q
             out[b, lo:hi, h] = sol_attn2_rows(q_bh[lo:hi], lo, k_bh, v_bh, r["mask"][i], counts, kg, vg,
                                               qbar_anchor)
     return dict(out=out, mask=masks)
+
+
+def dense_rows(q, k, v, q_start: int, q_tokens: int):
+    """Dense attention of the query tokens [q_start, q_start + q_tokens) over all keys (R17);
+    ``q_start < 0`` selects the suffix.  Returns FP64 [B, N, H, 128], NaN outside the rows."""
+    B, N, H, _ = q.shape
+    out = np.full((B, N, H, HEAD_DIM), np.nan)
+    if q_tokens <= 0:
+        return out
+    r0 = q_start if q_start >= 0 else N - q_tokens
+    r1 = min(N, r0 + q_tokens)
+    r0 = max(0, r0)
+    for b in range(B):
+        for h in range(H):
+            q_bh, k_bh, v_bh = head_slice(q, b, h), head_slice(k, b, h), head_slice(v, b, h)
+            z = SCALE * (q_bh[r0:r1] @ k_bh.T)
+            z -= z.max(axis=1, keepdims=True)
+            e = np.exp(z)
+            out[b, r0:r1, h] = (e @ v_bh) / e.sum(axis=1, keepdims=True)
+    return out
 
 
 def realised_sparsity(mask: np.ndarray) -> float:

@@ -67,3 +67,31 @@ def test_invalid_options_are_rejected_on_the_host(lib):
     opts = sa.Options(1)
     opts.reserved[3] = 1
     assert lib.sol_attn2_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa._options("exact", [(10, 0)])          # an extra sink needs tokens > 0
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa._options("exact", [(128, 4)])         # start must be < N
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa.Options()
+    opts.n_extra_sinks = 5                          # more than SOL_MAX_EXTRA_SINKS
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa.Options()
+    opts.extra_sink_tokens[2] = 3                   # an unused slot must stay zero
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    with pytest.raises(ValueError):
+        sa._options("exact", [(0, 1)] * 5)
+
+
+def test_options_struct_matches_the_header():
+    text = open(HEADER).read()
+    assert "#define SOL_MAX_EXTRA_SINKS 4" in text and sa.MAX_EXTRA_SINKS == 4
+    assert ctypes.sizeof(sa.Options) == 16 * 4
+
+
+def test_dense_rows_host_validation(lib):
+    rows = lambda **kw: lib.sol_attn_dense_rows(kw.get("q", 16), 16, 16, kw.get("out", 1 << 40), 1, kw.get("N", 128), 2,
+                                                kw.get("qs", 0), kw.get("qt", 10), None)
+    assert rows(q=0) == -1
+    assert rows(N=0) == -2
+    assert rows(qs=128) == -4          # q_start >= N
+    assert rows(q=17) == -5
+    assert rows(qt=0) == 0             # no rows: nothing to do, no device needed

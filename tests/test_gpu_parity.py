@@ -172,3 +172,44 @@ def test_diagonal_threshold_estimator(name):
     compare_outputs(out.float().cpu().numpy(), ref["out"], w.N, skip_rows=skip)
     exact = orc.routing(q, k, tau, w.sink_start, w.sink_tokens)
     assert not np.array_equal(exact["mask"], full["mask"])   # the estimator changes the routing
+
+
+@pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
+def test_extra_sink_ranges(entry):
+    """Several exact key ranges (the main sink plus extra ranges from the options) against the oracle."""
+    B, N, H, tau = 1, 3000, 2, 2.0
+    extra = [(900, 30), (2100, 200), (2990, 50)]
+    q, k, v = iid_qkv(B, N, H, seed=77)
+    fn = orc.sol_attn if entry == "sol_attn" else orc.sol_attn2
+    ref = fn(q, k, v, tau, 0, 100, extra_sinks=extra)
+    full = orc.routing(q, k, tau, 0, 100, extra_sinks=extra)
+    ref.update(shat=full["shat"], thresh=full["thresh"])
+    qd, kd, vd = _to_gpu(q, k, v)
+    gfn = sa.sol_attn_fwd if entry == "sol_attn" else sa.sol_attn2_fwd
+    out = gfn(qd, kd, vd, tau, 0, 100, extra_sinks=extra)
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    gmask, _ = sa.debug_route(qd, kd, tau, 0, 100, extra_sinks=extra)
+    flags = orc.sink_block_flags(N, 0, 100, extra)
+    assert flags.sum() >= 7
+    skip = check_mask(gmask.cpu().numpy(), ref, sink_flags=flags)
+    compare_outputs(out.float().cpu().numpy(), ref["out"], N, skip_rows=skip)
+
+
+@pytest.mark.parametrize("rows", [(70, 131), (0, 64), (-1, 40), (1500, 10_000)])
+def test_dense_rows_companion(rows):
+    """sol_attn_dense_rows: the given query rows get dense attention, every other row is untouched."""
+    B, N, H = 1, 2000, 2
+    q, k, v = iid_qkv(B, N, H, seed=91)
+    qd, kd, vd = _to_gpu(q, k, v)
+    out = sa.sol_attn_fwd(qd, kd, vd, 1.0, 0, 128)
+    before = out.clone()
+    sa.sol_attn_dense_rows(qd, kd, vd, out, rows[0], rows[1])
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    ref = orc.dense_rows(q, k, v, rows[0], rows[1])
+    sel = ~np.isnan(ref[0, :, 0, 0])
+    assert sel.any()
+    compare_outputs(out.float().cpu().numpy(), ref, N)
+    untouched = torch.from_numpy(~sel).to(out.device)
+    assert torch.equal(out[0][untouched], before[0][untouched])

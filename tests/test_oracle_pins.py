@@ -304,3 +304,38 @@ def test_diagonal_estimator_drops_channel_correlation():
     va = a.var()
     assert sig_d[0] == pytest.approx(S * np.sqrt(2 * va), rel=1e-12)
     assert sig_e[0] == pytest.approx(S * np.sqrt(4 * va), rel=1e-12)
+
+
+# ---------------------------------------------------- several sink ranges and dense text rows (R16, R17)
+
+def test_several_sink_ranges_hand_computed():
+    # N = 1000: blocks of 64 tokens, the last one (960..999) partial.  Tokens 100..129 touch blocks
+    # 1 and 2; token 700 lies in block 10; 990..1039 clips to 990..999 in block 15; the suffix of 5
+    # tokens (995..999) is block 15 again.
+    flags = orc.sink_block_flags(1000, -1, 5, extra_sinks=[(100, 30), (700, 1), (990, 50)])
+    assert sorted(np.nonzero(flags)[0].tolist()) == [1, 2, 10, 15]
+    assert not orc.sink_block_flags(1000, -1, 0, extra_sinks=[(5, 0)]).any()
+
+
+def test_extra_sinks_force_exact_columns_for_every_row():
+    q, k, _ = rand_qkv(1, 640, 1, seed=11)
+    r = orc.routing(q, k, tau=3.0, sink_start=0, sink_tokens=64, extra_sinks=[(300, 10), (600, 40)])
+    m = r["mask"][0, 0]
+    assert m[:, [0, 4, 9]].all()     # blocks 0 (0..63), 4 (256..319), 9 (576..639)
+
+
+def test_dense_rows_match_library_attention():
+    q, k, v = rand_qkv(1, 300, 2, seed=5)
+    out = orc.dense_rows(q, k, v, 70, 81)
+    ref = dense_attention(q, k, v)
+    np.testing.assert_allclose(out[:, 70:151], ref[:, 70:151], rtol=0, atol=1e-12)
+    assert np.isnan(out[:, :70]).all() and np.isnan(out[:, 151:]).all()
+    suf = orc.dense_rows(q, k, v, -1, 20)
+    np.testing.assert_allclose(suf[:, 280:], ref[:, 280:], rtol=0, atol=1e-12)
+
+
+def test_dense_rows_with_identical_keys_average_the_values():
+    q, k, v = rand_qkv(1, 130, 1, seed=6)
+    k[:] = k[:, :1]
+    out = orc.dense_rows(q, k, v, 0, 130)
+    np.testing.assert_allclose(out[0, :, 0], np.broadcast_to(v[0, :, 0].mean(axis=0), (130, D)), rtol=0, atol=1e-12)
