@@ -44,6 +44,8 @@ def parse_args():
                     help="heads (all query blocks each) the CPU oracle baseline evaluates")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--kv-splits", type=int, default=1,
+                    help="split-KV shares per 128-row query tile (Sol-Attn only; 1 = off)")
     return ap.parse_args()
 
 
@@ -274,8 +276,10 @@ def main():
     fn = sa.sol_attn_fwd if w.entry == "sol_attn" else sa.sol_attn2_fwd
     stream = torch.cuda.current_stream()
 
+    extra = {"kv_splits": args.kv_splits} if args.kv_splits != 1 else {}
+
     def step():
-        fn(q, k, v, tau, w.sink_start, w.sink_tokens, out=out, stream=stream)
+        fn(q, k, v, tau, w.sink_start, w.sink_tokens, out=out, stream=stream, **extra)
 
     for _ in range(args.warmup):
         step()
@@ -360,7 +364,7 @@ def main():
                                    if w.grid else w.name,
                        "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "tau": tau,
                        "target_sparsity": w.target_sparsity, "realised_sparsity": sp,
-                       "union_tile_useful_fraction": union_frac,
+                       "union_tile_useful_fraction": union_frac, "kv_splits": args.kv_splits,
                        "parallelism": f"independent replicas x{world} (head/batch sharding, no exchange)",
                        "l2": "inputs 1.6 GB per rank > 126 MB L2; no flush"},
             "frac_of_peak": value / world / peak_burst, "frac_of_sustained_peak": value / world / peak_sust,

@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libsolattn.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
-SOURCES = ["api.cu", "summary.cu", "route_tc.cu", "attn_fwd.cu", "sol2_tail.cu", "sol2_tail_tc.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "summary.cu", "route_tc.cu", "attn_fwd.cu", "splitkv.cu", "sol2_tail.cu", "sol2_tail_tc.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -250,10 +250,14 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   return check_launch("routing kernels");
 }
 
-// Validates the options against the sequence length; sets *diag.
-int check_options(const sol_attn_options* o, int N, bool* diag) {
+// Validates the options against the sequence length; sets *diag and *splits.
+int check_options(const sol_attn_options* o, int N, bool* diag, int* splits) {
   *diag = false;
+  *splits = 1;
   if (!o) return SOL_OK;
+  if (o->kv_splits < 0 || o->kv_splits > SOL_MAX_KV_SPLITS)
+    return fail(SOL_ERR_OPTION, "kv_splits must be in [0, %d]", SOL_MAX_KV_SPLITS);
+  *splits = o->kv_splits > 1 ? o->kv_splits : 1;
   for (int r : o->reserved)
     if (r != 0) return fail(SOL_ERR_OPTION, "reserved option fields must be zero");
   if (o->thresh_type != SOL_THRESH_EXACT && o->thresh_type != SOL_THRESH_DIAG)
@@ -276,7 +280,9 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   int rc = validate(q, k, v, out, true, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
   bool diag;
-  if ((rc = check_options(opts, N, &diag))) return rc;
+  int splits;
+  if ((rc = check_options(opts, N, &diag, &splits))) return rc;
+  if (sol2 && splits > 1) return fail(SOL_ERR_OPTION, "kv_splits > 1 is available for Sol-Attn only");
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;
   int dev;
@@ -284,9 +290,14 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   if ((rc = get_encode())) return rc;
   const Shape s = make_shape(B, N, H);
   Work w;
-  const size_t need = carve(s, sol2, nullptr, nullptr);
-  if ((rc = ensure_workspace(*d, need))) return rc;
+  const size_t base = carve(s, sol2, nullptr, nullptr);
+  const size_t rows_bh = (size_t)s.BH * s.QT * 128;
+  const size_t part_o_bytes = splits > 1 ? (size_t)splits * rows_bh * 128 * 4 : 0;
+  const size_t part_ml_bytes = splits > 1 ? (size_t)splits * rows_bh * 2 * 4 : 0;
+  if ((rc = ensure_workspace(*d, base + part_o_bytes + part_ml_bytes))) return rc;
   carve(s, sol2, static_cast<char*>(d->ws), &w);
+  float* part_o = splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(d->ws) + base) : nullptr;
+  float* part_ml = splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(d->ws) + base + part_o_bytes) : nullptr;
   w.stats = d->stats;
 
   CUtensorMap maps[5];
@@ -330,14 +341,23 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   p.tail_logz = w.tail_logz;
   p.tail_mu = w.tail_mu;
   p.tail_nu = w.tail_nu;
+  p.kv_splits = splits;
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.part_rows_bh = rows_bh;
   const int slot = d->timed_calls % DeviceState::kRing;
   if (g_timing) {
     if (!d->t0[slot] && (cudaEventCreate(&d->t0[slot]) != cudaSuccess || cudaEventCreate(&d->t1[slot]) != cudaSuccess))
       return fail(SOL_ERR_LAUNCH, "timing event creation failed");
     cudaEventRecord(d->t0[slot], st);
   }
-  cudaError_t e = launch_attn_fwd(maps, p, s.BH * s.QT, sol2, st);
+  cudaError_t e = launch_attn_fwd(maps, p, s.BH * s.QT * splits, sol2, st);
   if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "fused attention launch: %s", cudaGetErrorString(e));
+  if (splits > 1) {
+    launch_splitkv_combine(s, splits, part_o, part_ml, p.out, 0, N, st);
+    launches += 1;
+    if ((rc = check_launch("split-KV combine"))) return rc;
+  }
   if (g_timing) {
     cudaEventRecord(d->t1[slot], st);
     ++d->timed_calls;
@@ -394,6 +414,7 @@ int dense_rows(const void* q, const void* k, const void* v, void* out, int B, in
   p.qt_count = qt1 - qt0 + 1;
   p.row_lo = (int)r0;
   p.row_hi = (int)r1;
+  p.kv_splits = 1;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = d->status;
   cudaError_t e = launch_attn_fwd(maps, p, s.BH * p.qt_count, false, st);
@@ -404,6 +425,22 @@ int dense_rows(const void* q, const void* k, const void* v, void* out, int B, in
   d->last_launches = 2;
   g_last_device = dev;
   return SOL_OK;
+}
+
+// Self-test of the bounded-wait path: one thread waits on an mbarrier whose phase never completes
+// (nothing arrives on it), so the wait runs out after kWaitLimitNs and records a timeout in the
+// device status word exactly as a stalled pipeline stage would.  No trap, no fault: the kernel
+// returns normally and the context stays usable.
+__global__ void wait_timeout_selftest_kernel(int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag)) atomicExch(status, kDevTimeout);
 }
 
 }  // namespace
@@ -467,7 +504,8 @@ int sol_attn_debug_route_ex(const void* q, const void* k, int B, int N, int H, f
   int rc = validate(q, k, nullptr, nullptr, false, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
   bool diag;
-  if ((rc = check_options(opts, N, &diag))) return rc;
+  int splits;
+  if ((rc = check_options(opts, N, &diag, &splits))) return rc;
   if (!mask) return fail(SOL_ERR_NULL, "mask must be non-NULL");
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;
@@ -578,6 +616,20 @@ int sol_attn_dense_rows(const void* q, const void* k, const void* v, void* out, 
                         int q_tokens, void* stream) {
   g_err[0] = 0;
   return dense_rows(q, k, v, out, B, N, H, q_start, q_tokens, stream);
+}
+
+int sol_attn_selftest_wait_timeout(void* stream) {
+  g_err[0] = 0;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* d;
+  int dev;
+  int rc = device_state(&d, &dev);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(d->status);
+  if ((rc = check_launch("wait-timeout self-test"))) return rc;
+  d->last_stream = st;
+  return SOL_OK;
 }
 
 }  // extern "C"

@@ -65,6 +65,7 @@ struct __align__(1024) FwdSmem {
   float xm[2][128], xl[2][128];   // [warpgroup][row] running max and row sum, for the epilogue merge
   uint32_t tmem_base;
   int abort;
+  int tile_lo, tile_hi;     // this CTA's share [tile_lo, tile_hi) of the unit's tile list
 };
 
 // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (checked at run time: a
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(384, 1)
   FwdSmem& sm = *reinterpret_cast<FwdSmem*>(smem_raw);
   volatile int* abort = &sm.abort;
 
-  const int unit = (int)blockIdx.x;
+  const int unit = (int)blockIdx.x / p.kv_splits, split = (int)blockIdx.x % p.kv_splits;
   const int bh = unit / p.qt_count, qt = p.qt_begin + unit % p.qt_count;
   const int b = bh / p.H, h = bh % p.H;
   const int qb0 = 2 * qt;
@@ -155,14 +156,54 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
+  if (warp == 2) {
+    // the unit's tile count (exact pairs over the union of its two rows, then surrogate chunks),
+    // split into kv_splits contiguous shares; one share for the whole list without split-KV
+    int lo = 0, hi = 0x7fffffff;
+    if (p.kv_splits > 1) {
+      const uint32_t* row0 = p.mask + ((size_t)bh * p.Nb + qb0) * p.Nw;
+      const uint32_t* row1 = row0 + p.Nw;
+      int uni = 0, pooled_tiles = 0;
+      for (int wd = lane; wd < p.Nw; wd += 32) {
+        const uint32_t a = row0[wd], c = has_hi ? row1[wd] : 0u;
+        uni += __popc(a | c);
+      }
+      if (!kSol2) {
+        for (int ch = lane; ch < (p.Nb + 127) / 128; ch += 32) {
+          bool any = false;
+          for (int e = 0; e < 4; ++e) {
+            const int wd = 4 * ch + e;
+            if (wd >= p.Nw) break;
+            const int nvalid = min(32, p.Nb - 32 * wd);
+            const uint32_t valid = nvalid >= 32 ? 0xffffffffu : ((1u << nvalid) - 1u);
+            if ((~row0[wd] & valid) || (has_hi && (~row1[wd] & valid))) any = true;
+          }
+          pooled_tiles += any ? 1 : 0;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        uni += __shfl_xor_sync(0xffffffffu, uni, o);
+        pooled_tiles += __shfl_xor_sync(0xffffffffu, pooled_tiles, o);
+      }
+      const int total = (uni + 1) / 2 + pooled_tiles;
+      lo = (int)((long long)total * split / p.kv_splits);
+      hi = (int)((long long)total * (split + 1) / p.kv_splits);
+    }
+    if (lane == 0) {
+      sm.tile_lo = lo;
+      sm.tile_hi = hi;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const bool empty_share = sm.tile_lo >= sm.tile_hi;   // split-KV: no key tile for this CTA
 
   if (warp == 0) {
     // ----------------------------------------------------------------------------------- producer
-    if (lane == 0) {
+    if (lane == 0 && !empty_share) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -204,7 +245,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         ++t;
       };
+      int g = 0;   // index of the next tile in the unit's list (split-KV keeps [tile_lo, tile_hi))
+      const int g_lo = sm.tile_lo, g_hi = sm.tile_hi;
       auto push = [&](TileDesc d) {
+        const int gi = g++;
+        if (gi < g_lo || gi >= g_hi) return;
         if (have_prev && ok) issue(prev);
         prev = d;
         have_prev = true;
@@ -259,7 +304,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 1) {
     // --------------------------------------------------------------------------- S = Q K^T issuer
-    if (lane == 0) {
+    if (lane == 0 && !empty_share) {
       bool ok = mbar_wait(&sm.qfull, 0, abort);
       const uint32_t q_base = smem_u32(&sm.q[0][0]);
       for (int t = 0; ok; ++t) {
@@ -297,7 +342,7 @@ __global__ void __launch_bounds__(384, 1)
     // One product per softmax warpgroup and tile: O_w += P_w V_w over the warpgroup's 64 keys, issued
     // as soon as that warpgroup's P is in TMEM.  A separate thread from the Q K^T issuer, so neither
     // queues behind the other in program order.
-    if (lane == 0) {
+    if (lane == 0 && !empty_share) {
       bool ok = true;
       bool b_started = false;
       for (int u = 0; ok; ++u) {
@@ -342,7 +387,7 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------------------------ V producer
     // Loads V tiles in the order the K producer published them, so that K tiles (needed first, by
     // Q K^T) never wait behind the release of a V stage.
-    if (lane == 0) {
+    if (lane == 0 && !empty_share) {
       bool ok = true;
       int u = 0;
       for (;; ++u) {
@@ -394,6 +439,13 @@ __global__ void __launch_bounds__(384, 1)
     const float lg_last = log2f((float)n_last);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    if (empty_share) {
+      if (wg == 0 && row_valid) {
+        const size_t prow = (size_t)(blockIdx.x % p.kv_splits) * p.part_rows_bh + (size_t)bh * p.QT * 128 + tok;
+        p.part_ml[2 * prow] = -INFINITY;   // no key in this share: weight 0 in the combine
+        p.part_ml[2 * prow + 1] = 0.f;
+      }
+    } else {
     bool o1_written = false;   // O_1 receives a product for every tile with a second 64-key half
     int t = 0;
     for (;; ++t) {
@@ -584,7 +636,28 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld_wait();
       const float ws = (self_written && w_self > 0.f) ? w_self * scale_o : 0.f;
       const float wo = (other_written && w_other > 0.f) ? w_other * scale_o : 0.f;
-      if (row_valid) {
+      if (p.kv_splits > 1) {
+        // split-KV: the partial state of this share (O relative to the merged reference m_ref)
+        if (row_valid) {
+          const size_t prow = (size_t)(blockIdx.x % p.kv_splits) * p.part_rows_bh + (size_t)bh * p.QT * 128 + tok;
+          float* dst = p.part_o + prow * 128 + 64 * wg;
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            float o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float a = w_self > 0.f ? __uint_as_float(oa[c + e]) * w_self : 0.f;
+              if (w_other > 0.f) a = fmaf(__uint_as_float(ob[c + e]), w_other, a);
+              o4[e] = a;
+            }
+            *reinterpret_cast<float4*>(dst + c) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+          }
+          if (wg == 0) {
+            p.part_ml[2 * prow] = m_ref;
+            p.part_ml[2 * prow + 1] = l_tot;
+          }
+        }
+      } else if (row_valid) {
         __nv_bfloat16* orow = p.out + ((size_t)((size_t)b * p.N + tok) * p.H + h) * 128 + 64 * wg;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
@@ -608,6 +681,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
+    }   // non-empty share
   }
   tc_fence_before();
   __syncthreads();

@@ -13,6 +13,13 @@ struct FwdParams {
   int qt_begin, qt_count;    // query tiles (pairs of query blocks) qt_begin .. + qt_count - 1 of each (b, h)
   int row_lo, row_hi;        // token rows [row_lo, row_hi) are written; the others are computed only
   __nv_bfloat16* out;        // [B][N][H][128]
+  // split-KV (kv_splits > 1): CTA s of a query tile takes the s-th contiguous share of its key
+  // tiles and writes its partial state instead of `out`: part_o [kv_splits][BH][QT * 128][128]
+  // (unnormalised O relative to the row's base-2 reference), part_ml [...][2] = (reference, sum)
+  int kv_splits;
+  float* part_o;
+  float* part_ml;
+  size_t part_rows_bh;       // BH * QT * 128: rows of one split's partial state
   int* status;               // device status word
   // Sol-Attn2 tail (unused by Sol-Attn)
   const float* qanchor;      // [BH][Na][128]

@@ -79,6 +79,9 @@ struct SinkSet {
   int n;
   int b0[kMaxSinkRanges], b1[kMaxSinkRanges];
 };
+// Split-KV combine (splitkv.cu): merges the kv_splits partial states of every query row into out.
+void launch_splitkv_combine(const Shape& s, int splits, const float* part_o, const float* part_ml,
+                            __nv_bfloat16* out, int row_lo, int row_hi, cudaStream_t st);
 cudaError_t launch_route_tc(const void* maps, const Shape& s, const Work& w, const SinkSet& sinks, int* status,
                             cudaStream_t st);
 void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, cudaStream_t st);

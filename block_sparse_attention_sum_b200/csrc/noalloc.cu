@@ -215,6 +215,7 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   p.qt_count = s.QT;
   p.row_lo = 0;
   p.row_hi = N;
+  p.kv_splits = 1;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = d.status;
   cudaError_t e = launch_attn_fwd(maps, p, s.BH * s.QT, false, st);

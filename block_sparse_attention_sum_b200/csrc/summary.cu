@@ -134,12 +134,29 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
 // -------------------------------------------------------------------------------------------------
 constexpr int kGramSplits = 8;
 
-__global__ void kmean_kernel(Shape s, Work w) {
-  const int bh = blockIdx.x, c = threadIdx.x;
-  const float* kb = w.kbar + (size_t)bh * s.Nb * kHeadDim;
-  double acc = 0.0;
-  for (int j = 0; j < s.Nb; ++j) acc += (double)kb[(size_t)j * kHeadDim + c];
-  w.kmean[(size_t)bh * kHeadDim + c] = acc / s.Nb;
+// kmean: 8 row groups of 128 threads (thread = channel) sum every 8th key block with four
+// independent FP64 accumulators each, then the groups combine in shared memory.
+__global__ void __launch_bounds__(1024) kmean_kernel(Shape s, Work w) {
+  __shared__ double part[8][kHeadDim];
+  const int bh = blockIdx.x, c = threadIdx.x & (kHeadDim - 1), g = threadIdx.x >> 7;
+  const float* kb = w.kbar + (size_t)bh * s.Nb * kHeadDim + c;
+  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  int j = g;
+  for (; j + 24 < s.Nb; j += 32) {
+    a0 += (double)kb[(size_t)j * kHeadDim];
+    a1 += (double)kb[(size_t)(j + 8) * kHeadDim];
+    a2 += (double)kb[(size_t)(j + 16) * kHeadDim];
+    a3 += (double)kb[(size_t)(j + 24) * kHeadDim];
+  }
+  for (; j < s.Nb; j += 8) a0 += (double)kb[(size_t)j * kHeadDim];
+  part[g][c] = (a0 + a1) + (a2 + a3);
+  __syncthreads();
+  if (g == 0) {
+    double acc = 0.0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc += part[e][c];
+    w.kmean[(size_t)bh * kHeadDim + c] = acc / s.Nb;
+  }
 }
 
 __global__ void __launch_bounds__(256) kgram_kernel(Shape s, Work w, float* partial) {
@@ -308,7 +325,7 @@ void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_b
 }
 
 void launch_kstats(const Shape& s, const Work& w, cudaStream_t st) {
-  kmean_kernel<<<s.BH, kHeadDim, 0, st>>>(s, w);
+  kmean_kernel<<<s.BH, 8 * kHeadDim, 0, st>>>(s, w);
   kgram_kernel<<<dim3(kGramSplits, s.BH), 256, 0, st>>>(s, w, w.gram_partial);
   kgram_reduce_kernel<<<dim3(kHeadDim * kHeadDim / 256, s.BH), 256, 0, st>>>(s, w, w.gram_partial);
 }

@@ -34,6 +34,7 @@ EXPORTS = [
     "sol_attn_release_workspace",
     "sol_attn_fwd_noalloc",
     "sol_attn_dense_rows",
+    "sol_attn_selftest_wait_timeout",
 ]
 
 STATUS = {
@@ -44,6 +45,7 @@ STATUS = {
 
 THRESH_TYPES = {"exact": 0, "diag": 1}
 MAX_EXTRA_SINKS = 4
+MAX_KV_SPLITS = 8
 
 
 class Options(ctypes.Structure):
@@ -51,11 +53,12 @@ class Options(ctypes.Structure):
 
     _fields_ = [("thresh_type", ctypes.c_int), ("n_extra_sinks", ctypes.c_int),
                 ("extra_sink_start", ctypes.c_int * MAX_EXTRA_SINKS), ("extra_sink_tokens", ctypes.c_int * MAX_EXTRA_SINKS),
-                ("reserved", ctypes.c_int * 6)]
+                ("kv_splits", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
 
 
-def _options(thresh_type: str, extra_sinks=()):
-    """extra_sinks: up to MAX_EXTRA_SINKS (start, tokens) token ranges made exact for every query."""
+def _options(thresh_type: str, extra_sinks=(), kv_splits: int = 1):
+    """extra_sinks: up to MAX_EXTRA_SINKS (start, tokens) token ranges made exact for every query;
+    kv_splits: split-KV shares per query tile (1 = off)."""
     if thresh_type not in THRESH_TYPES:
         raise ValueError(f"thresh_type must be one of {sorted(THRESH_TYPES)}")
     extra_sinks = list(extra_sinks)
@@ -64,6 +67,7 @@ def _options(thresh_type: str, extra_sinks=()):
     o = Options()
     o.thresh_type = THRESH_TYPES[thresh_type]
     o.n_extra_sinks = len(extra_sinks)
+    o.kv_splits = int(kv_splits)
     for e, (start, tokens) in enumerate(extra_sinks):
         o.extra_sink_start[e] = int(start)
         o.extra_sink_tokens[e] = int(tokens)
@@ -126,6 +130,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_fwd_noalloc.restype = i
     lib.sol_attn_dense_rows.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.sol_attn_dense_rows.restype = i
+    lib.sol_attn_selftest_wait_timeout.argtypes = [vp]
+    lib.sol_attn_selftest_wait_timeout.restype = i
     _lib = lib
     return lib
 
@@ -154,7 +160,8 @@ def _check_qkv(q, k, v=None):
     return q.shape[0], q.shape[1], q.shape[2]
 
 
-def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type="exact", extra_sinks=()):
+def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type="exact", extra_sinks=(),
+         kv_splits=1):
     B, N, H = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
@@ -164,8 +171,8 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
     args = [q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, float(tau), int(sink_start),
             int(sink_tokens)]
     with torch.cuda.device(q.device):
-        if thresh_type != "exact" or extra_sinks:
-            opts = _options(thresh_type, extra_sinks)
+        if thresh_type != "exact" or extra_sinks or kv_splits != 1:
+            opts = _options(thresh_type, extra_sinks, kv_splits)
             rc = getattr(lib, fn_name + "_ex")(*args, ctypes.byref(opts), _stream_handle(stream))
         else:
             rc = getattr(lib, fn_name)(*args, _stream_handle(stream))
@@ -174,9 +181,10 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
 
 
 def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
-                 extra_sinks=()):
+                 extra_sinks=(), kv_splits=1):
     """Sol-Attn forward through the C ABI; returns ``out`` (BF16 [B, N, H, 128])."""
-    return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks)
+    return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks,
+                kv_splits)
 
 
 def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
@@ -238,6 +246,11 @@ def last_stats():
     mn, mx = ctypes.c_int(), ctypes.c_int()
     _check(lib.sol_attn_last_stats(ctypes.byref(e), ctypes.byref(t), ctypes.byref(mn), ctypes.byref(mx)))
     return e.value, t.value, mn.value, mx.value
+
+
+def selftest_wait_timeout(stream=None) -> int:
+    """Enqueue the bounded-wait self-test (see include/sol_attn.h); returns its launch status."""
+    return load_library().sol_attn_selftest_wait_timeout(_stream_handle(stream))
 
 
 def get_device_status(stream=None) -> int:

@@ -63,6 +63,7 @@ typedef enum {
 } sol_thresh_type;
 
 #define SOL_MAX_EXTRA_SINKS 4
+#define SOL_MAX_KV_SPLITS 8
 
 /*
  * Options of the _ex entry points.  A NULL pointer means all defaults (an all-zero struct is the
@@ -74,13 +75,22 @@ typedef enum {
  *                      tokens [extra_sink_start[e], extra_sink_start[e] + extra_sink_tokens[e]),
  *                      clipped to N; it needs 0 <= start < N and tokens > 0.  Like the main sink,
  *                      every key block overlapping a range is exact for every query.
+ *   kv_splits          0 or 1: one CTA per 128-row query tile.  2 .. SOL_MAX_KV_SPLITS: split-KV
+ *                      (the Sol-Attn README's kv_splits, "Long-sequence tuning on H100"): each
+ *                      query tile's key tiles are divided into kv_splits contiguous shares, one CTA
+ *                      each, and a combine kernel merges the partial softmax states exactly
+ *                      (o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s).  Results equal the
+ *                      unsplit call up to FP32 rounding.  Raises parallelism when there are few
+ *                      query tiles; the workspace grows by kv_splits * B*H*ceil(N/128)*128 * 520
+ *                      bytes.  Sol-Attn only: sol_attn2_fwd_ex rejects kv_splits > 1.
  */
 typedef struct {
   int thresh_type;
   int n_extra_sinks;
   int extra_sink_start[SOL_MAX_EXTRA_SINKS];
   int extra_sink_tokens[SOL_MAX_EXTRA_SINKS];
-  int reserved[6];
+  int kv_splits;
+  int reserved[5];
 } sol_attn_options;
 
 /*
@@ -205,6 +215,17 @@ int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
  */
 int sol_attn_dense_rows(const void* q, const void* k, const void* v, void* out, int B, int N, int H, int q_start,
                         int q_tokens, void* stream);
+
+/*
+ * Self-test of the device-side failure path (no counterpart on the pages; for tests and health
+ * checks).  Enqueues on `stream` one tiny kernel whose single bounded wait can never be satisfied,
+ * so it runs out after about one second and records a timeout in the device status word, as a
+ * stalled pipeline stage in the attention kernels would.  Nothing traps or faults; the next
+ * sol_attn_get_device_status(stream) returns SOL_ERR_TIMEOUT (and clears the word), after which
+ * the library works as before.  Returns SOL_OK once enqueued, or SOL_ERR_DEVICE without a usable
+ * device.
+ */
+int sol_attn_selftest_wait_timeout(void* stream);
 
 #ifdef __cplusplus
 }

@@ -79,11 +79,16 @@ def test_invalid_options_are_rejected_on_the_host(lib):
     assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
     with pytest.raises(ValueError):
         sa._options("exact", [(0, 1)] * 5)
+    opts = sa._options("exact", kv_splits=9)        # more than SOL_MAX_KV_SPLITS
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa._options("exact", kv_splits=-1)
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
 
 
 def test_options_struct_matches_the_header():
     text = open(HEADER).read()
     assert "#define SOL_MAX_EXTRA_SINKS 4" in text and sa.MAX_EXTRA_SINKS == 4
+    assert "#define SOL_MAX_KV_SPLITS 8" in text and sa.MAX_KV_SPLITS == 8
     assert ctypes.sizeof(sa.Options) == 16 * 4
 
 

@@ -213,3 +213,32 @@ def test_dense_rows_companion(rows):
     compare_outputs(out.float().cpu().numpy(), ref, N)
     untouched = torch.from_numpy(~sel).to(out.device)
     assert torch.equal(out[0][untouched], before[0][untouched])
+
+
+@pytest.mark.parametrize("kv_splits", [2, 4, 8])
+@pytest.mark.parametrize("case", [("n129", 1, 129, 2, 1.0, -1, 0), ("n1000_b2", 2, 1000, 2, 1.0, -1, 0),
+                                  ("n4000_high_tau", 1, 4000, 2, 3.0, -1, 0)], ids=lambda c: c[0])
+def test_split_kv(case, kv_splits):
+    """kv_splits > 1 (README "Long-sequence tuning"): shares of each query tile's key tiles on separate
+    CTAs, merged by the combine kernel; the same oracle result (n129 with 8 splits leaves most shares
+    empty)."""
+    name, B, N, H, tau, ss, st = case
+    q, k, v = _small_inputs(name, B, N, H)
+    ref = orc.sol_attn(q, k, v, tau, ss, st)
+    qd, kd, vd = _to_gpu(q, k, v)
+    out = sa.sol_attn_fwd(qd, kd, vd, tau, ss, st, kv_splits=kv_splits)
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    assert sa.last_launch_count() == 8   # routing (6) + fused kernel + combine
+    gmask, _ = sa.debug_route(qd, kd, tau, ss, st)
+    skip = check_mask(gmask.cpu().numpy(), ref)
+    compare_outputs(out.float().cpu().numpy(), ref["out"], N, skip_rows=skip)
+    one = sa.sol_attn_fwd(qd, kd, vd, tau, ss, st)
+    torch.cuda.synchronize()
+    assert (out.float() - one.float()).abs().max().item() <= 1.6e-2
+
+
+def test_split_kv_is_sol_attn_only():
+    q, k, v = _to_gpu(*iid_qkv(1, 256, 1, seed=3))
+    with pytest.raises(sa.SolAttnError):
+        sa._fwd("sol_attn2_fwd", q, k, v, 1.0, -1, 0, None, None, "exact", (), 2)
