@@ -632,4 +632,31 @@ int sol_attn_selftest_wait_timeout(void* stream) {
   return SOL_OK;
 }
 
+int sol_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, const int* cu_seqlens, int nseq,
+                        int H, float tau, int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream) {
+  g_err[0] = 0;
+  if (!cu_seqlens) return fail(SOL_ERR_NULL, "cu_seqlens must be non-NULL");
+  if (nseq <= 0 || H <= 0) return fail(SOL_ERR_SHAPE, "nseq and H must be positive");
+  if (cu_seqlens[0] != 0) return fail(SOL_ERR_SHAPE, "cu_seqlens[0] must be 0");
+  for (int i = 0; i < nseq; ++i)
+    if (cu_seqlens[i + 1] < cu_seqlens[i]) return fail(SOL_ERR_SHAPE, "cu_seqlens must be non-decreasing");
+  // every sequence must satisfy the single-sequence rules (a sink range starts inside each one)
+  for (int i = 0; i < nseq; ++i) {
+    const int n = cu_seqlens[i + 1] - cu_seqlens[i];
+    if (n > 0 && sink_tokens > 0 && sink_start >= n)
+      return fail(SOL_ERR_SINK, "sink_start (%d) must be < the length of sequence %d (%d)", sink_start, i, n);
+  }
+  const size_t row = (size_t)H * 128 * 2;   // bytes per token
+  for (int i = 0; i < nseq; ++i) {
+    const int n = cu_seqlens[i + 1] - cu_seqlens[i];
+    if (n == 0) continue;
+    const size_t off = (size_t)cu_seqlens[i] * row;
+    const int rc = forward(static_cast<const char*>(q) + off, static_cast<const char*>(k) + off,
+                           static_cast<const char*>(v) + off, static_cast<char*>(out) + off, 1, n, H, tau, sink_start,
+                           sink_tokens, opts, stream, false);
+    if (rc) return rc;
+  }
+  return SOL_OK;
+}
+
 }  // extern "C"

@@ -33,6 +33,7 @@ EXPORTS = [
     "sol_attn_last_launch_count",
     "sol_attn_release_workspace",
     "sol_attn_fwd_noalloc",
+    "sol_attn_fwd_varlen",
     "sol_attn_dense_rows",
     "sol_attn_selftest_wait_timeout",
 ]
@@ -130,6 +131,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_fwd_noalloc.restype = i
     lib.sol_attn_dense_rows.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.sol_attn_dense_rows.restype = i
+    lib.sol_attn_fwd_varlen.argtypes = [vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int), i, i, f, i, i, op, vp]
+    lib.sol_attn_fwd_varlen.restype = i
     lib.sol_attn_selftest_wait_timeout.argtypes = [vp]
     lib.sol_attn_selftest_wait_timeout.restype = i
     _lib = lib
@@ -191,6 +194,30 @@ def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stre
                   extra_sinks=()):
     """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
     return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks)
+
+
+def sol_attn_fwd_varlen(q, k, v, cu_seqlens, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None,
+                        thresh_type="exact", extra_sinks=(), kv_splits=1):
+    """Packed variable-length batch: q, k, v BF16 [total_tokens, H, 128]; sequence s is the tokens
+    cu_seqlens[s] .. cu_seqlens[s + 1] - 1 (a host list of offsets starting at 0)."""
+    for t in (q, k, v):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 3 \
+                or t.shape[-1] != HEAD_DIM or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v must be contiguous BF16 CUDA tensors [total_tokens, H, 128] of one shape")
+    if out is None:
+        out = torch.empty_like(q)
+    cu = [int(x) for x in cu_seqlens]
+    if cu[-1] > q.shape[0]:
+        raise ValueError("cu_seqlens exceeds the packed token count")
+    arr = (ctypes.c_int * len(cu))(*cu)
+    opts = _options(thresh_type, extra_sinks, kv_splits)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.sol_attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), arr, len(cu) - 1,
+                                     q.shape[1], float(tau), int(sink_start), int(sink_tokens), ctypes.byref(opts),
+                                     _stream_handle(stream))
+    _check(rc)
+    return out
 
 
 def sol_attn_dense_rows(q, k, v, out, q_start, q_tokens, stream=None):

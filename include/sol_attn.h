@@ -201,6 +201,21 @@ int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
                          int sink_start, int sink_tokens, void* stream);
 
 /*
+ * Variable-length batch (packed sequences, as the pages' integrations pass them): sequence s holds
+ * the tokens [cu_seqlens[s], cu_seqlens[s + 1]) of the packed tensors q, k, v, out, each laid out
+ * [total_tokens, H, 128] (BTHD with B = 1 per sequence).  Every sequence is an independent
+ * sol_attn_fwd_ex call on its own tokens (its own blocks, thresholds and routing; the sink range
+ * and extra sinks are relative to each sequence's first token), issued in order on `stream`.
+ *   cu_seqlens : HOST int array of nseq + 1 non-decreasing offsets, cu_seqlens[0] = 0; empty
+ *                sequences are skipped.  Pointers and options follow sol_attn_fwd_ex.
+ *   Errors: SOL_ERR_NULL / SOL_ERR_SHAPE for a bad cu_seqlens, SOL_ERR_SINK when sink_start is not
+ *   inside every non-empty sequence; otherwise the first failing sequence's status (earlier
+ *   sequences are already enqueued).  sol_attn_last_stats then reports the last sequence.
+ */
+int sol_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, const int* cu_seqlens, int nseq,
+                        int H, float tau, int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream);
+
+/*
  * Dense companion call for text query rows in joint (MMDiT) attention.  The Sol-Attn README,
  * "Exact KV sink": a sink keeps the text KEY blocks exact for every query but does not make the
  * text QUERY rows dense; an integration should use dense attention for the valid text queries and

@@ -100,3 +100,16 @@ def test_dense_rows_host_validation(lib):
     assert rows(qs=128) == -4          # q_start >= N
     assert rows(q=17) == -5
     assert rows(qt=0) == 0             # no rows: nothing to do, no device needed
+
+
+def test_varlen_host_validation(lib):
+    import ctypes as C
+    arr = lambda xs: (C.c_int * len(xs))(*xs)
+    opts = sa.Options()
+    call = lambda cu, n, ss=-1, st=0: lib.sol_attn_fwd_varlen(16, 16, 16, 1 << 40, cu, n, 2, 1.0, ss, st, C.byref(opts), None)
+    assert call(None, 1) == -1
+    assert call(arr([0, 10]), 0) == -2
+    assert call(arr([1, 10]), 1) == -2           # must start at 0
+    assert call(arr([0, 10, 5]), 2) == -2        # non-decreasing
+    assert call(arr([0, 100, 150]), 2, ss=60, st=4) == -4   # the sink start lies beyond sequence 1
+    assert call(arr([0, 0, 0]), 2) == 0          # only empty sequences: nothing to do

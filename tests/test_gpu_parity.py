@@ -242,3 +242,27 @@ def test_split_kv_is_sol_attn_only():
     q, k, v = _to_gpu(*iid_qkv(1, 256, 1, seed=3))
     with pytest.raises(sa.SolAttnError):
         sa._fwd("sol_attn2_fwd", q, k, v, 1.0, -1, 0, None, None, "exact", (), 2)
+
+
+def test_varlen_packed_batch():
+    """sol_attn_fwd_varlen: packed sequences of different lengths (one empty), each against the oracle
+    on its own tokens, with a per-sequence prefix sink."""
+    H, tau = 2, 1.0
+    lens = [700, 0, 64, 1300]
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    q, k, v = iid_qkv(1, cu[-1], H, seed=55)
+    out = sa.sol_attn_fwd_varlen(*(t[0].cuda() for t in (q, k, v)), cu, tau, 0, 32)
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    got = out.float().cpu().numpy()
+    for s, n in enumerate(lens):
+        if n == 0:
+            continue
+        sl = slice(cu[s], cu[s + 1])
+        qs, ks, vs = q[:, sl], k[:, sl], v[:, sl]
+        ref = orc.sol_attn(qs, ks, vs, tau, 0, 32)
+        gmask, _ = sa.debug_route(qs.cuda(), ks.cuda(), tau, 0, 32)
+        skip = check_mask(gmask.cpu().numpy(), ref)
+        compare_outputs(got[None, sl], ref["out"], n, skip_rows=skip)

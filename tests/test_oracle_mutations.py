@@ -63,6 +63,29 @@ def _suffix_off_by_one(N, sink_start, sink_tokens):
 _orig_sink = orc.sink_block_flags
 
 
+def _extra_sinks_ignored(N, sink_start, sink_tokens, extra_sinks=()):
+    return _orig_sink(N, sink_start, sink_tokens)
+
+
+_orig_dense = orc.dense_rows
+
+
+def _dense_rows_one_short(q, k, v, q_start, q_tokens):
+    return _orig_dense(q, k, v, q_start, q_tokens - 1)
+
+
+def _dense_rows_unscaled(q, k, v, q_start, q_tokens):
+    return _orig_dense(q / orc.SCALE, k, v, q_start, q_tokens)
+
+
+_orig_diag = orc.threshold_diag
+
+
+def _diag_without_mean(Qbar, Kbar, tau):
+    mu, sigma, thresh = _orig_diag(Qbar, Kbar, tau)
+    return 0.0 * mu, sigma, tau * sigma
+
+
 CASES = [
     ("block_sums", _value_means_not_sums,
      lambda: pins.test_identical_unselected_keys_make_the_approximation_exact(448, "sol_attn")),
@@ -79,6 +102,10 @@ CASES = [
     ("sink_block_flags", _suffix_off_by_one, pins.test_sink_blocks_by_hand),
     ("SCALE", 1.0, lambda: pins.test_sink_over_everything_is_dense_attention(200, "sol_attn")),
     ("SCALE", 2.0 * orc.SCALE, pins.test_hand_expanded_sol_attn),
+    ("sink_block_flags", _extra_sinks_ignored, pins.test_several_sink_ranges_hand_computed),
+    ("dense_rows", _dense_rows_one_short, pins.test_dense_rows_match_library_attention),
+    ("dense_rows", _dense_rows_unscaled, pins.test_dense_rows_match_library_attention),
+    ("threshold_diag", _diag_without_mean, pins.test_diagonal_estimator_equals_exact_when_key_covariance_is_diagonal),
 ]
 
 
