@@ -133,15 +133,22 @@ size_t carve(const Shape& s, bool sol2, char* base, Work* w) {
   return off;
 }
 
+// Upper bound on the workspace of one device (0: none); lets callers cap the library's memory and
+// lets tests exercise the allocation-failure path without exhausting a GPU.
+size_t g_ws_limit = 0;
+
 int ensure_workspace(DeviceState& d, size_t bytes) {
   if (d.ws_bytes >= bytes) return SOL_OK;
+  if (g_ws_limit && bytes > g_ws_limit)
+    return fail(SOL_ERR_ALLOC, "workspace of %zu bytes exceeds the limit of %zu bytes", bytes, g_ws_limit);
   if (d.ws) {
     cudaDeviceSynchronize();
     cudaFree(d.ws);
     d.ws = nullptr;
     d.ws_bytes = 0;
   }
-  const size_t grow = align_up(bytes + bytes / 8, 1 << 20);
+  size_t grow = align_up(bytes + bytes / 8, 1 << 20);
+  if (g_ws_limit && grow > g_ws_limit) grow = bytes;
   if (cudaMalloc(&d.ws, grow) != cudaSuccess) {
     cudaGetLastError();
     return fail(SOL_ERR_ALLOC, "workspace allocation of %zu bytes failed", grow);
@@ -494,6 +501,7 @@ int sol_attn_get_device_status(void* stream) {
     return fail(SOL_ERR_LAUNCH, "status read failed");
   if (h == kDevTimeout) return fail(SOL_ERR_TIMEOUT, "a bounded wait inside a kernel ran out");
   if (h == kDevMisaligned) return fail(SOL_ERR_LAUNCH, "shared memory window misaligned; the kernel did not run");
+  if (h == kDevBounds) return fail(SOL_ERR_LAUNCH, "a bounds check of the debug build failed (access skipped)");
   return SOL_OK;
 }
 
@@ -657,6 +665,11 @@ int sol_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, 
     if (rc) return rc;
   }
   return SOL_OK;
+}
+
+void sol_attn_set_workspace_limit(size_t bytes) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_ws_limit = bytes;
 }
 
 }  // extern "C"

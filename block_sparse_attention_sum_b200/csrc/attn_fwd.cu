@@ -109,6 +109,21 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 
 __device__ __forceinline__ void set_timeout(int* status) { atomicExch(status, kDevTimeout); }
 
+// Debug builds (-DSOL_ATTN_DEBUG_BOUNDS) check every TMA tile coordinate against the tensor it
+// reads; a failed check records kDevBounds in the status word and the copy is skipped (its consumer
+// then runs out its bounded wait).  Release builds compile the checks away.
+__device__ __forceinline__ bool tile_ok(uint32_t kind, int j0, int j1, int Nb, int* status) {
+#ifdef SOL_ATTN_DEBUG_BOUNDS
+  const bool ok = kind == 2u ? (j0 >= 0 && 128 * j0 < Nb)
+                             : (j0 >= 0 && j0 < Nb && (kind != 0u || (j1 > j0 && j1 < Nb)));
+  if (!ok) atomicExch(status, kDevBounds);
+  return ok;
+#else
+  (void)kind; (void)j0; (void)j1; (void)Nb; (void)status;
+  return true;
+#endif
+}
+
 }  // namespace
 
 template <bool kSol2>
@@ -212,6 +227,7 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_desc(&tm_vp);
       }
       mbar_arrive_expect_tx(&sm.qfull, 4 * kBoxBytes);
+      if (tile_ok(1u, qb0, 0, p.Nb, p.status))
       for (int hf = 0; hf < 2; ++hf)
         for (int dh = 0; dh < 2; ++dh)
           tma_load_4d(&sm.q[dh][hf * 64 * 64], &tm_q, &sm.qfull, 64 * dh, h, 64 * (qb0 + hf), b);
@@ -235,7 +251,8 @@ __global__ void __launch_bounds__(384, 1)
         const int nblk = d.kind == kTilePair ? 2 : 1;
         const uint32_t bytes = pooled ? 2 * kTileBytes : 2 * kBoxBytes * nblk;
         mbar_arrive_expect_tx(&sm.kfull[s], bytes);
-        if (pooled) {
+        if (!tile_ok(d.kind, d.j0, d.j1, p.Nb, p.status)) {
+        } else if (pooled) {
           for (int dh = 0; dh < 2; ++dh) tma_load_3d(&sm.k[s][dh][0], &tm_kp, &sm.kfull[s], 64 * dh, 128 * d.j0, bh);
         } else {
           for (int slot = 0; slot < nblk; ++slot)
@@ -401,7 +418,8 @@ __global__ void __launch_bounds__(384, 1)
         const bool pooled = d.kind == kTilePooled;
         const int nblk = d.kind == kTilePair ? 2 : 1;
         mbar_arrive_expect_tx(&sm.vfull[s], pooled ? 2 * kTileBytes : 2 * kBoxBytes * nblk);
-        if (pooled) {
+        if (!tile_ok(d.kind, d.j0, d.j1, p.Nb, p.status)) {
+        } else if (pooled) {
           for (int dh = 0; dh < 2; ++dh) tma_load_3d(&sm.v[s][dh][0], &tm_vp, &sm.vfull[s], 64 * dh, 128 * d.j0, bh);
         } else {
           for (int slot = 0; slot < nblk; ++slot)

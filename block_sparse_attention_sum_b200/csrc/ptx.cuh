@@ -13,6 +13,7 @@ enum : int {
   kDevOk = 0,
   kDevTimeout = 1,
   kDevMisaligned = 2,   // dynamic shared memory not 1024-byte aligned
+  kDevBounds = 3,       // debug build: an index check failed and the access was skipped
 };
 
 // Upper bound on any single mbarrier wait, in nanoseconds of %globaltimer (about one second).

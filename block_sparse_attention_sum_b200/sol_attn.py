@@ -35,6 +35,7 @@ EXPORTS = [
     "sol_attn_fwd_noalloc",
     "sol_attn_fwd_varlen",
     "sol_attn_dense_rows",
+    "sol_attn_set_workspace_limit",
     "sol_attn_selftest_wait_timeout",
 ]
 
@@ -133,6 +134,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_dense_rows.restype = i
     lib.sol_attn_fwd_varlen.argtypes = [vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int), i, i, f, i, i, op, vp]
     lib.sol_attn_fwd_varlen.restype = i
+    lib.sol_attn_set_workspace_limit.argtypes = [ctypes.c_size_t]
+    lib.sol_attn_set_workspace_limit.restype = None
     lib.sol_attn_selftest_wait_timeout.argtypes = [vp]
     lib.sol_attn_selftest_wait_timeout.restype = i
     _lib = lib
@@ -299,6 +302,11 @@ def kernel_ms_sum(n: int) -> float:
 
 def last_launch_count() -> int:
     return int(load_library().sol_attn_last_launch_count())
+
+
+def set_workspace_limit(nbytes: int):
+    """Cap the library's per-device workspace (0 removes the cap); see include/sol_attn.h."""
+    load_library().sol_attn_set_workspace_limit(int(nbytes))
 
 
 def release_workspace():

@@ -38,6 +38,8 @@
 #ifndef SOL_ATTN_H_
 #define SOL_ATTN_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -230,6 +232,15 @@ int sol_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, 
  */
 int sol_attn_dense_rows(const void* q, const void* k, const void* v, void* out, int B, int N, int H, int q_start,
                         int q_tokens, void* stream);
+
+/*
+ * Caps the workspace the library may hold on each device at `bytes` (0 removes the cap; applies to
+ * later calls).  A call that would need more returns SOL_ERR_ALLOC with a message and launches
+ * nothing; an existing larger workspace is kept until sol_attn_release_workspace().  No counterpart
+ * on the pages: it bounds the library's memory next to other users of the GPU and makes the
+ * allocation-failure path testable.
+ */
+void sol_attn_set_workspace_limit(size_t bytes);
 
 /*
  * Self-test of the device-side failure path (no counterpart on the pages; for tests and health
