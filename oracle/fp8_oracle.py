@@ -1,0 +1,133 @@
+"""FP64 reference for the FP8 (E4M3) + ExpCast variant of the Sol-Attn forward.
+
+TEST INFRASTRUCTURE ONLY, like ``sol_attn_oracle``: only the tests (and the bench's CPU legs) may
+import it; the product path never does.  It shares no code with the CUDA path.
+
+Source: "Sol-Attn2: Sparse Attention with Complementary Approximation", section "FP8 quantization
+and ExpCast":
+
+* Q and K are quantised with one E4M3 scale per 64-token block, V with one scale per head: for a
+  nonzero block X, s_X = max|X| / 448, X_8 = FP8_E4M3(X / s_X), X ~= s_X X_8.
+* QK and PV use the FP8 operands with FP32 accumulation; the scales restore the magnitudes.
+* ExpCast turns a base-2 score directly into an E4M3 probability byte: with a shared online pivot m,
+  u = (s - m) log2 e, c(u) = clip_[0,120](RNE(8u + 55.65)), p(u) = decode_E4M3(c(u)) ~= 2^u.  The same
+  decoded weights enter the PV product and the denominator.
+
+Readings (also listed in the design notes):
+
+R18 The FP8 path quantises the operands of the exact branch (token-level Q K^T and P V); routing
+    (block means, thresholds, masks) and the surrogate operands (block means of K, value sums) stay
+    as in the BF16 path, computed from the original inputs.
+R19 ExpCast gives every weight of the shared softmax, exact tokens and surrogate blocks alike (the
+    surrogate's log-mass ln n_j is part of its score, as in the BF16 path); numerator and denominator
+    use the same decoded weights.  The oracle's pivot is the row maximum, so u <= 0; a kernel pivot
+    that lags the maximum by at most 8 (base 2) stays inside the code range (c = 120 is u ~ 8.04).
+R20 An all-zero quantisation block keeps scale 1 and zero codes.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from oracle import sol_attn_oracle as orc
+
+E4M3_MAX = 448.0
+EXPCAST_OFFSET = 55.65
+EXPCAST_MAX_CODE = 120
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Round to the nearest E4M3 value (ties to even), saturating at +-448.
+
+    E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; normal values (1 + m/8) 2^(e-7)
+    for e = 1..15 (largest finite 1.75 * 2^8 = 448), subnormals m 2^-9."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))           # binade, at least the smallest normal one
+    step = 2.0 ** (e - 3)                                      # 3 mantissa bits (2^-9 for subnormals)
+    r = np.round(a / step) * step                              # numpy rounds half to even
+    return np.sign(x) * np.minimum(r, E4M3_MAX)
+
+
+def e4m3_decode(code) -> np.ndarray:
+    """Value of non-negative E4M3 codes 0..126 (bit pattern 0 eeee mmm)."""
+    c = np.asarray(code, dtype=np.int64)
+    e, m = c >> 3, c & 7
+    return np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+
+
+def expcast_code(u) -> np.ndarray:
+    """c(u) = clip_[0,120](RNE(8u + 55.65))."""
+    return np.clip(np.round(8.0 * np.asarray(u, dtype=np.float64) + EXPCAST_OFFSET), 0, EXPCAST_MAX_CODE).astype(np.int64)
+
+
+def expcast(u) -> np.ndarray:
+    """p(u) = decode_E4M3(c(u)) ~= 2^u."""
+    return e4m3_decode(expcast_code(u))
+
+
+def quantize(x) -> tuple[np.ndarray, float]:
+    """One E4M3 scale for the whole array: (s_X X_8 as FP64, s_X)."""
+    x = np.asarray(x, dtype=np.float64)
+    amax = float(np.abs(x).max()) if x.size else 0.0
+    s = amax / E4M3_MAX if amax > 0 else 1.0
+    return s * e4m3_round(x / s), s
+
+
+def quantize_blocks(x_bh: np.ndarray, block: int = orc.BLOCK) -> np.ndarray:
+    """Per 64-token block of one head's [N, 128] rows (the last block partial): dequantised E4M3."""
+    out = np.empty_like(np.asarray(x_bh, dtype=np.float64))
+    for j in range(orc.num_blocks(x_bh.shape[0])):
+        a, b = orc.block_range(j, x_bh.shape[0])
+        out[a:b] = quantize(x_bh[a:b])[0]
+    return out
+
+
+def sol_attn_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat, counts, q_rows):
+    """Outputs of one query block's rows under the FP8 path.
+
+    Exact tokens: logits from the dequantised E4M3 operands (FP64 here; FP32 accumulation in the
+    kernel), values from the dequantised V.  Surrogate blocks: logits q.Kbar_j / sqrt(d) from the
+    original query rows plus ln n_j, values Vhat_j / n_j per unit of mass.  Every weight is ExpCast of
+    its base-2 score against the row maximum (R19)."""
+    N = k8_bh.shape[0]
+    ex = np.nonzero(mask_row)[0]
+    un = np.nonzero(~mask_row)[0]
+    tok = np.concatenate([np.arange(*orc.block_range(j, N)) for j in ex]) if len(ex) else np.zeros(0, np.int64)
+    z = orc.SCALE * (q8_rows @ k8_bh[tok].T)
+    logmass = orc.SCALE * (q_rows @ Kbar[un].T) + np.log(counts[un].astype(np.float64))[None, :]
+    M = np.full(q_rows.shape[0], -np.inf)
+    if z.shape[1]:
+        M = np.maximum(M, z.max(axis=1))
+    if logmass.shape[1]:
+        M = np.maximum(M, logmass.max(axis=1))
+    pz = expcast((z - M[:, None]) / math.log(2.0))
+    pa = expcast((logmass - M[:, None]) / math.log(2.0))
+    vbar = Vhat[un] / counts[un][:, None]
+    num = pz @ v8_bh[tok] + pa @ vbar
+    den = pz.sum(axis=1) + pa.sum(axis=1)
+    return num / den[:, None]
+
+
+def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None):
+    """FP8 + ExpCast Sol-Attn forward.  Returns dict with ``out`` (FP64, NaN for rows not computed)
+    and ``mask`` (the routing of the BF16 path, R18)."""
+    B, N, H, _ = q.shape
+    Nb = orc.num_blocks(N)
+    sink = orc.sink_block_flags(N, sink_start, sink_tokens)
+    out = np.full((B, N, H, orc.HEAD_DIM), np.nan)
+    masks = np.zeros((B, H, Nb, Nb), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            q_bh, k_bh, v_bh = orc.head_slice(q, b, h), orc.head_slice(k, b, h), orc.head_slice(v, b, h)
+            r = orc._routing_for_head(q_bh, k_bh, tau, sink)
+            masks[b, h] = r["mask"]
+            q8, k8 = quantize_blocks(q_bh), quantize_blocks(k_bh)
+            v8 = quantize(v_bh)[0]
+            Vhat = orc.block_sums(v_bh)
+            for i in (range(Nb) if qblocks is None else qblocks):
+                lo, hi = orc.block_range(i, N)
+                out[b, lo:hi, h] = sol_attn_fp8_rows(q8[lo:hi], k8, v8, r["mask"][i], r["Kbar"], Vhat, r["counts"],
+                                                     q_bh[lo:hi])
+    return dict(out=out, mask=masks)

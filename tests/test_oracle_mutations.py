@@ -114,3 +114,47 @@ def test_planted_mistake_is_caught(monkeypatch, name, broken, pin):
     monkeypatch.setattr(orc, name, broken)
     with pytest.raises(AssertionError):
         pin()
+
+
+# ---------------------------------------------------------------- FP8 + ExpCast reference
+from oracle import fp8_oracle as f8  # noqa: E402
+from tests import test_oracle_fp8 as fp8pins  # noqa: E402
+
+
+def _decode_bias_8(code):
+    c = np.asarray(code, dtype=np.int64)
+    e, m = c >> 3, c & 7
+    return np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 8.0))
+
+
+def _expcast_no_clip(u):
+    return f8.e4m3_decode(np.maximum(np.round(8.0 * np.asarray(u, dtype=np.float64) + f8.EXPCAST_OFFSET), 0).astype(np.int64))
+
+
+def _quantize_no_scale(x):
+    x = np.asarray(x, dtype=np.float64)
+    return f8.e4m3_round(x), 1.0
+
+
+_orig_fp8_rows = f8.sol_attn_fp8_rows
+
+
+def _fp8_surrogate_sums(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat, counts, q_rows):
+    return _orig_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat * counts[:, None], counts, q_rows)
+
+
+FP8_CASES = [
+    ("e4m3_decode", _decode_bias_8, fp8pins.test_e4m3_decode_matches_torch),
+    ("expcast_code", lambda u: np.round(8.0 * np.asarray(u) + f8.EXPCAST_OFFSET).astype(np.int64),
+     fp8pins.test_expcast_powers_of_two_and_error_bound),
+    ("expcast", _expcast_no_clip, fp8pins.test_expcast_powers_of_two_and_error_bound),
+    ("quantize", _quantize_no_scale, fp8pins.test_quantizer_extremes),
+    ("sol_attn_fp8_rows", _fp8_surrogate_sums, fp8pins.test_fp8_forward_with_zero_queries_averages_the_values),
+]
+
+
+@pytest.mark.parametrize("name,broken,pin", FP8_CASES, ids=[f"fp8-{c[0]}-{i}" for i, c in enumerate(FP8_CASES)])
+def test_planted_fp8_mistake_is_caught(monkeypatch, name, broken, pin):
+    monkeypatch.setattr(f8, name, broken)
+    with pytest.raises(AssertionError):
+        pin()
