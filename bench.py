@@ -22,6 +22,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -132,7 +133,8 @@ class ClockSampler:
 
     def __init__(self, device_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = os.path.join(os.environ.get("SOL_BENCH_CLOCKS_DIR", tempfile.gettempdir()),
+                                 f"sol_bench_clocks_rank{device_index}.csv")
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")

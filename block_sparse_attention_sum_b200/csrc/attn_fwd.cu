@@ -7,7 +7,7 @@
 // one online-softmax state, K/V loaded only for routed blocks; pooled key KC and summed value VC).
 // Sol-Attn2 draft, "Routing and complementary approximation" (tail merged in the epilogue).
 //
-// B200 design (differs from the paper's nested loop, see the design notes):
+// B200 design (it differs from the paper's nested loop):
 //  * A work unit is a 128-row query tile = two adjacent 64-token query blocks, so every tcgen05.mma
 //    runs at M = 128.  The unit walks the union of the two blocks' exact sets, two key blocks
 //    (128 keys) per tile; columns of a block that is exact for only one half are masked for the

@@ -13,7 +13,7 @@ and ExpCast":
   u = (s - m) log2 e, c(u) = clip_[0,120](RNE(8u + 55.65)), p(u) = decode_E4M3(c(u)) ~= 2^u.  The same
   decoded weights enter the PV product and the denominator.
 
-Readings (also listed in the design notes):
+Readings:
 
 R18 The FP8 path quantises the operands of the exact branch (token-level Q K^T and P V); routing
     (block means, thresholds, masks) and the surrogate operands (block means of K, value sums) stay

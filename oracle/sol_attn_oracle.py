@@ -27,7 +27,7 @@ Sources (page title, section / equation):
 * [sdcpp]    stable-diffusion.cpp "Sol-Attn" documentation: adjacent blocks remain exact; K means
   and V sums for the approximate blocks; one shared online-softmax normaliser.
 
-Readings where the pages are silent, ambiguous or garbled (each is also listed in the design notes):
+Readings where the pages are silent, ambiguous or garbled:
 
 R1  Scale: s = 1/sqrt(128) on token logits, proxies, thresholds and surrogate logits ([Sol2] uses
     z = q.k/sqrt(d); the paper's Eqs. (1)-(3) print no scale).  The routing mask does not depend
