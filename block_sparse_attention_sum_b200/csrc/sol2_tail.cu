@@ -15,17 +15,28 @@ namespace sol {
 
 // u = mean of all queries of a (b, h) = sum_j n_j Qbar_j / N, accumulated in FP64.  Also marks the
 // padding groups 2 Nb .. Gp - 1 of the log-size row as empty.
-__global__ void qdir_kernel(Shape s, Work w) {
-  const int bh = blockIdx.x, c = threadIdx.x;
+// Eight row groups of 128 threads (thread = channel) sum every eighth block, then combine.
+__global__ void __launch_bounds__(1024) qdir_kernel(Shape s, Work w) {
+  __shared__ double part[8][kHeadDim];
+  const int bh = blockIdx.x, c = threadIdx.x & (kHeadDim - 1), g = threadIdx.x >> 7;
   const int gp = tail_groups_padded(s);
-  if (2 * s.Nb + c < gp) w.glog2n[(size_t)bh * gp + 2 * s.Nb + c] = -INFINITY;
-  const float* qb = w.qbar + (size_t)bh * s.Nb * kHeadDim;
-  double acc = 0.0;
-  for (int j = 0; j < s.Nb; ++j) {
-    const int n = min(kBlock, s.N - j * kBlock);
-    acc += (double)n * (double)qb[(size_t)j * kHeadDim + c];
+  if (g == 0 && 2 * s.Nb + c < gp) w.glog2n[(size_t)bh * gp + 2 * s.Nb + c] = -INFINITY;
+  const float* qb = w.qbar + (size_t)bh * s.Nb * kHeadDim + c;
+  double a0 = 0.0, a1 = 0.0;
+  int j = g;
+  for (; j + 8 < s.Nb; j += 16) {
+    a0 += (double)min(kBlock, s.N - j * kBlock) * (double)qb[(size_t)j * kHeadDim];
+    a1 += (double)min(kBlock, s.N - (j + 8) * kBlock) * (double)qb[(size_t)(j + 8) * kHeadDim];
   }
-  w.qdir[(size_t)bh * kHeadDim + c] = (float)(acc / s.N);
+  for (; j < s.Nb; j += 8) a0 += (double)min(kBlock, s.N - j * kBlock) * (double)qb[(size_t)j * kHeadDim];
+  part[g][c] = a0 + a1;
+  __syncthreads();
+  if (g == 0) {
+    double acc = 0.0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc += part[e][c];
+    w.qdir[(size_t)bh * kHeadDim + c] = (float)(acc / s.N);
+  }
 }
 
 // Two groups per key block: group 1 = keys with k.u > Kbar_j.u, group 0 = the rest (FP32 decision).
@@ -145,7 +156,7 @@ __global__ void __launch_bounds__(256) groups_kernel(const __nv_bfloat16* __rest
 void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
                    const Work& w, cudaStream_t st) {
   (void)q;
-  qdir_kernel<<<s.BH, kHeadDim, 0, st>>>(s, w);
+  qdir_kernel<<<s.BH, 8 * kHeadDim, 0, st>>>(s, w);
   groups_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(k, v, s, w);
 }
 

@@ -232,11 +232,31 @@ __global__ void __launch_bounds__(256) thresh_kernel(Shape s, Work w, float tau,
   const int bh = blockIdx.y, i0 = blockIdx.x * 64, tid = threadIdx.x;
   const float* cov = w.kcov + (size_t)bh * kHeadDim * kHeadDim;
   const float* qb = w.qbar + (size_t)bh * s.Nb * kHeadDim;
-  for (int idx = tid; idx < kHeadDim * kHeadDim / 4; idx += 256)
-    reinterpret_cast<float4*>(cov_s)[idx] = reinterpret_cast<const float4*>(cov)[idx];
-  for (int idx = tid; idx < 64 * kHeadDim; idx += 256) {
-    const int r = idx / kHeadDim, c = idx % kHeadDim;
-    qt[c * kThreshPad + r] = (i0 + r < s.Nb) ? qb[(size_t)(i0 + r) * kHeadDim + c] : 0.f;
+  // all global loads of a thread are issued before the first shared-memory store, so they are in
+  // flight together (16 x 16 bytes of the covariance, 8 x 16 bytes of the query-block means)
+  {
+    float4 cv[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) cv[e] = reinterpret_cast<const float4*>(cov)[tid + 256 * e];
+    // lane = row (so the transposed shared-memory stores of a warp hit 32 consecutive words),
+    // warp and e pick the four channels
+    float4 qv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int r = (tid & 31) + 32 * (e & 1), c4 = (tid >> 5) + 8 * (e >> 1);
+      qv[e] = (i0 + r < s.Nb) ? reinterpret_cast<const float4*>(qb + (size_t)(i0 + r) * kHeadDim)[c4]
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) reinterpret_cast<float4*>(cov_s)[tid + 256 * e] = cv[e];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int r = (tid & 31) + 32 * (e & 1), c = 4 * ((tid >> 5) + 8 * (e >> 1));
+      qt[(c + 0) * kThreshPad + r] = qv[e].x;
+      qt[(c + 1) * kThreshPad + r] = qv[e].y;
+      qt[(c + 2) * kThreshPad + r] = qv[e].z;
+      qt[(c + 3) * kThreshPad + r] = qv[e].w;
+    }
   }
   __syncthreads();
   if (tid < 64) {
