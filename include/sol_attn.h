@@ -142,7 +142,9 @@ const char* sol_attn_last_error(void);
 /*
  * Synchronises `stream`, then reads and clears this device's status word.  Returns SOL_OK, or
  * SOL_ERR_TIMEOUT if a bounded wait inside a kernel ran out since the last read, or
- * SOL_ERR_LAUNCH if the synchronisation itself failed.
+ * SOL_ERR_LAUNCH if the synchronisation itself failed, a kernel found its shared-memory window
+ * misaligned (it then returned without running), or a bounds check of the debug build
+ * (libsolattn_debug.so) failed and the access was skipped.
  */
 int sol_attn_get_device_status(void* stream);
 
@@ -166,7 +168,8 @@ int sol_attn_last_stats(long long* exact_pairs, long long* total_pairs, int* min
 
 /*
  * Kernel timing for measurement: when enabled (nonzero), each forward call records a pair of CUDA
- * events on its stream around the fused attention kernel, in a ring of 256 pairs per device that
+ * events on its stream around the fused attention kernel (and, with kv_splits > 1, the combine
+ * kernel that follows it), in a ring of 256 pairs per device that
  * enabling resets.  sol_attn_last_kernel_ms() synchronises on the most recent closing event and
  * returns that launch's duration in milliseconds; sol_attn_kernel_ms_sum(n) returns the summed
  * duration of the last n timed launches (n <= 256).  Both return a negative value if unavailable.
