@@ -20,8 +20,14 @@ R18 The FP8 path quantises the operands of the exact branch (token-level Q K^T a
     as in the BF16 path, computed from the original inputs.
 R19 ExpCast gives every weight of the shared softmax, exact tokens and surrogate blocks alike (the
     surrogate's log-mass ln n_j is part of its score, as in the BF16 path); numerator and denominator
-    use the same decoded weights.  The oracle's pivot is the row maximum, so u <= 0; a kernel pivot
-    that lags the maximum by at most 8 (base 2) stays inside the code range (c = 120 is u ~ 8.04).
+    use the same decoded weights.  The pivot is an integer in base 2: ExpCast is not invariant under
+    fractional shifts of u, but for an integer shift k the code moves by exactly 8k (one E4M3
+    binade), so weights coded against any integer pivot agree up to the factor 2^-k except below
+    2^-6 of the pivot (subnormal codes and the clip at 0).  The code range [0, 120] spans
+    u in [-6.96, 8.04]: a pivot at the maximum would leave half of it unused and drop every weight
+    below 2^-7 of the maximum, so the reference takes the pivot ceil(row max) - 8 in base 2
+    (u <= 8, the largest weight coded 112..120), the same range an online pivot moved only when the
+    running maximum exceeds it by more than 8 keeps.
 R20 An all-zero quantisation block keeps scale 1 and zero codes.
 """
 from __future__ import annotations
@@ -90,7 +96,7 @@ def sol_attn_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat, counts, q_row
     Exact tokens: logits from the dequantised E4M3 operands (FP64 here; FP32 accumulation in the
     kernel), values from the dequantised V.  Surrogate blocks: logits q.Kbar_j / sqrt(d) from the
     original query rows plus ln n_j, values Vhat_j / n_j per unit of mass.  Every weight is ExpCast of
-    its base-2 score against the row maximum (R19)."""
+    its base-2 score against the integer pivot ceil(row max / ln 2) - 8 (R19)."""
     N = k8_bh.shape[0]
     ex = np.nonzero(mask_row)[0]
     un = np.nonzero(~mask_row)[0]
@@ -102,8 +108,9 @@ def sol_attn_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat, counts, q_row
         M = np.maximum(M, z.max(axis=1))
     if logmass.shape[1]:
         M = np.maximum(M, logmass.max(axis=1))
-    pz = expcast((z - M[:, None]) / math.log(2.0))
-    pa = expcast((logmass - M[:, None]) / math.log(2.0))
+    pivot = np.ceil(M / math.log(2.0)) - 8.0                            # integer base-2 pivot
+    pz = expcast(z / math.log(2.0) - pivot[:, None])
+    pa = expcast(logmass / math.log(2.0) - pivot[:, None])
     vbar = Vhat[un] / counts[un][:, None]
     num = pz @ v8_bh[tok] + pa @ vbar
     den = pz.sum(axis=1) + pa.sum(axis=1)

@@ -77,10 +77,11 @@ def test_fp8_forward_reduces_to_the_bf16_path_without_rounding(monkeypatch):
 
 def test_fp8_forward_error_is_that_of_its_roundings():
     # with the roundings in place the result moves by about the E4M3 / ExpCast resolution (a few
-    # percent), not more
+    # percent: 5 % here), not more; a pivot at the row maximum instead of 8 binades below it would
+    # drop every weight under 2^-7 of the maximum and double the error
     g = np.random.default_rng(5)
     q, k, v = (g.standard_normal((1, 640, 1, 128)) for _ in range(3))
     a = f8.sol_attn_fp8(q, k, v, tau=1.0)["out"]
     b = orc.sol_attn(q, k, v, tau=1.0)["out"]
     rel = np.linalg.norm(a - b) / np.linalg.norm(b)
-    assert 0.005 < rel < 0.2, rel
+    assert 0.005 < rel < 0.1, rel
