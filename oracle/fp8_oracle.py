@@ -15,9 +15,15 @@ and ExpCast":
 
 Readings:
 
-R18 The FP8 path quantises the operands of the exact branch (token-level Q K^T and P V); routing
-    (block means, thresholds, masks) and the surrogate operands (block means of K, value sums) stay
-    as in the BF16 path, computed from the original inputs.
+R18 Both products of the shared softmax take FP8 operands (the section gives FP8 operands to QK and
+    PV and keeps the mass of the compressed keys by a bias added to their scores): the exact
+    branch's tokens as above, and the
+    surrogate's compressed keys and values under the same rules - the block means Kbar_j quantised
+    as a key array (one scale per 64 consecutive compressed keys of a head), the value means
+    Vbar_j = Vhat_j / n_j with the head's V scale (|Vbar| <= max |V|, so they stay in range).  A
+    surrogate block's logit is q8 . Kbar8_j / sqrt(d) plus the additive bias ln n_j, its value
+    Vbar8_j per unit of that mass.  Routing (block means, thresholds, masks) stays as in the BF16
+    path, computed from the original inputs.
 R19 ExpCast gives every weight of the shared softmax, exact tokens and surrogate blocks alike (the
     surrogate's log-mass ln n_j is part of its score, as in the BF16 path); numerator and denominator
     use the same decoded weights.  The pivot is an integer in base 2: ExpCast is not invariant under
@@ -90,20 +96,20 @@ def quantize_blocks(x_bh: np.ndarray, block: int = orc.BLOCK) -> np.ndarray:
     return out
 
 
-def sol_attn_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat, counts, q_rows):
+def sol_attn_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, kbar8, vbar8, counts):
     """Outputs of one query block's rows under the FP8 path.
 
     Exact tokens: logits from the dequantised E4M3 operands (FP64 here; FP32 accumulation in the
-    kernel), values from the dequantised V.  Surrogate blocks: logits q.Kbar_j / sqrt(d) from the
-    original query rows plus ln n_j, values Vhat_j / n_j per unit of mass.  Every weight is ExpCast of
-    its base-2 score against the integer pivot ceil(row max / ln 2) - 8 (R19)."""
+    kernel), values from the dequantised V.  Surrogate blocks: logits q8 . Kbar8_j / sqrt(d) plus
+    ln n_j, values Vbar8_j per unit of mass (R18).  Every weight is ExpCast of its base-2 score
+    against the integer pivot ceil(row max / ln 2) - 8 (R19)."""
     N = k8_bh.shape[0]
     ex = np.nonzero(mask_row)[0]
     un = np.nonzero(~mask_row)[0]
     tok = np.concatenate([np.arange(*orc.block_range(j, N)) for j in ex]) if len(ex) else np.zeros(0, np.int64)
     z = orc.SCALE * (q8_rows @ k8_bh[tok].T)
-    logmass = orc.SCALE * (q_rows @ Kbar[un].T) + np.log(counts[un].astype(np.float64))[None, :]
-    M = np.full(q_rows.shape[0], -np.inf)
+    logmass = orc.SCALE * (q8_rows @ kbar8[un].T) + np.log(counts[un].astype(np.float64))[None, :]
+    M = np.full(q8_rows.shape[0], -np.inf)
     if z.shape[1]:
         M = np.maximum(M, z.max(axis=1))
     if logmass.shape[1]:
@@ -111,10 +117,17 @@ def sol_attn_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat, counts, q_row
     pivot = np.ceil(M / math.log(2.0)) - 8.0                            # integer base-2 pivot
     pz = expcast(z / math.log(2.0) - pivot[:, None])
     pa = expcast(logmass / math.log(2.0) - pivot[:, None])
-    vbar = Vhat[un] / counts[un][:, None]
-    num = pz @ v8_bh[tok] + pa @ vbar
+    num = pz @ v8_bh[tok] + pa @ vbar8[un]
     den = pz.sum(axis=1) + pa.sum(axis=1)
     return num / den[:, None]
+
+
+def surrogate_operands_fp8(Kbar, Vhat, counts, v_scale: float):
+    """E4M3 compressed keys and values of one head (R18): Kbar per 64 consecutive block means,
+    Vbar = Vhat / n with the head's V scale."""
+    kbar8 = quantize_blocks(Kbar)
+    vbar = Vhat / counts[:, None]
+    return kbar8, v_scale * e4m3_round(vbar / v_scale)
 
 
 def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None):
@@ -131,10 +144,9 @@ def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0
             r = orc._routing_for_head(q_bh, k_bh, tau, sink)
             masks[b, h] = r["mask"]
             q8, k8 = quantize_blocks(q_bh), quantize_blocks(k_bh)
-            v8 = quantize(v_bh)[0]
-            Vhat = orc.block_sums(v_bh)
+            v8, sv = quantize(v_bh)
+            kbar8, vbar8 = surrogate_operands_fp8(r["Kbar"], orc.block_sums(v_bh), r["counts"], sv)
             for i in (range(Nb) if qblocks is None else qblocks):
                 lo, hi = orc.block_range(i, N)
-                out[b, lo:hi, h] = sol_attn_fp8_rows(q8[lo:hi], k8, v8, r["mask"][i], r["Kbar"], Vhat, r["counts"],
-                                                     q_bh[lo:hi])
+                out[b, lo:hi, h] = sol_attn_fp8_rows(q8[lo:hi], k8, v8, r["mask"][i], kbar8, vbar8, r["counts"])
     return dict(out=out, mask=masks)

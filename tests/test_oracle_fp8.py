@@ -52,15 +52,34 @@ def test_quantizer_extremes():
 
 def test_fp8_forward_with_zero_queries_averages_the_values():
     # q = 0: every exact token has score 0 and every surrogate block log-mass ln 64, so ExpCast gives
-    # 2^-6 per token and 1 per block exactly; with V on the E4M3 grid the output is the mean of V.
+    # 2^-6 per token and 1 per block exactly; with V constant over each block and on the E4M3 grid of
+    # its head scale (so that the block means are too), the output is the mean of V.
     N, H = 512, 2
     g = np.random.default_rng(3)
     q = np.zeros((1, N, H, 128))
     k = g.standard_normal((1, N, H, 128))
-    v = g.choice([-1.0, -0.5, 0.0, 0.5, 1.0], size=(1, N, H, 128))
-    v[0, 0, :, 0] = 1.0
+    vb = g.choice([-1.0, -0.5, 0.0, 0.5, 1.0], size=(1, N // 64, H, 128))
+    vb[0, 0, :, 0] = 1.0
+    v = np.repeat(vb, 64, axis=1)
     out = f8.sol_attn_fp8(q, k, v, tau=1.0)["out"]
     np.testing.assert_allclose(out[0], np.broadcast_to(v[0].mean(axis=0), (N, H, 128)), rtol=0, atol=1e-12)
+
+
+def test_surrogate_operands_are_quantised_like_keys_and_values():
+    # compressed keys: one scale per 64 consecutive block means; compressed values: the head's V scale
+    g = np.random.default_rng(6)
+    Kbar = g.standard_normal((150, 128))
+    Kbar[64:128] *= 100.0                                              # a second group 100x larger
+    counts = np.full(150, 64)
+    counts[-1] = 17
+    Vhat = g.standard_normal((150, 128)) * counts[:, None]
+    kbar8, vbar8 = f8.surrogate_operands_fp8(Kbar, Vhat, counts, v_scale=0.01)
+    for a, b in ((0, 64), (64, 128), (128, 150)):
+        s = np.abs(Kbar[a:b]).max() / 448.0
+        np.testing.assert_array_equal(kbar8[a:b], s * f8.e4m3_round(Kbar[a:b] / s))
+    vbar = Vhat / counts[:, None]
+    np.testing.assert_array_equal(vbar8, 0.01 * f8.e4m3_round(vbar / 0.01))
+    assert np.abs(vbar8 - vbar).max() <= 2.0 ** -4 * np.abs(vbar).max()
 
 
 def test_fp8_forward_reduces_to_the_bf16_path_without_rounding(monkeypatch):

@@ -139,8 +139,21 @@ def _quantize_no_scale(x):
 _orig_fp8_rows = f8.sol_attn_fp8_rows
 
 
-def _fp8_surrogate_sums(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat, counts, q_rows):
-    return _orig_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, Kbar, Vhat * counts[:, None], counts, q_rows)
+def _fp8_surrogate_sums(q8_rows, k8_bh, v8_bh, mask_row, kbar8, vbar8, counts):
+    return _orig_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, kbar8, vbar8 * counts[:, None], counts)
+
+
+def _surrogate_one_key_scale(Kbar, Vhat, counts, v_scale):
+    _, vbar8 = _orig_surrogate(Kbar, Vhat, counts, v_scale)
+    return f8.quantize(Kbar)[0], vbar8
+
+
+def _surrogate_sums_quantised(Kbar, Vhat, counts, v_scale):
+    kbar8, _ = _orig_surrogate(Kbar, Vhat, counts, v_scale)
+    return kbar8, v_scale * f8.e4m3_round(Vhat / v_scale)
+
+
+_orig_surrogate = f8.surrogate_operands_fp8
 
 
 FP8_CASES = [
@@ -150,6 +163,12 @@ FP8_CASES = [
     ("expcast", _expcast_no_clip, fp8pins.test_expcast_powers_of_two_and_error_bound),
     ("quantize", _quantize_no_scale, fp8pins.test_quantizer_extremes),
     ("sol_attn_fp8_rows", _fp8_surrogate_sums, fp8pins.test_fp8_forward_with_zero_queries_averages_the_values),
+    ("surrogate_operands_fp8", _surrogate_one_key_scale,
+     fp8pins.test_surrogate_operands_are_quantised_like_keys_and_values),
+    ("surrogate_operands_fp8", _surrogate_sums_quantised,
+     fp8pins.test_surrogate_operands_are_quantised_like_keys_and_values),
+    ("surrogate_operands_fp8", _surrogate_sums_quantised,
+     fp8pins.test_fp8_forward_with_zero_queries_averages_the_values),
 ]
 
 
