@@ -17,7 +17,8 @@ LIB_NAME = "libsolattn.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 # the same library with the device-side bounds checks compiled in (-DSOL_ATTN_DEBUG_BOUNDS)
 DEBUG_LIB_PATH = os.path.join(HERE, "libsolattn_debug.so")
-SOURCES = ["api.cu", "summary.cu", "route_tc.cu", "attn_fwd.cu", "splitkv.cu", "sol2_tail.cu", "sol2_tail_tc.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "summary.cu", "route_tc.cu", "attn_fwd.cu", "splitkv.cu", "sol2_tail.cu", "sol2_tail_tc.cu", "noalloc.cu",
+           "quant_fp8.cu", "attn_fwd_fp8.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -13,6 +13,8 @@
 #include <vector>
 
 #include "attn_fwd.cuh"
+#include "attn_fwd_fp8.cuh"
+#include "fp8.cuh"
 #include "common.cuh"
 #include "ptx.cuh"
 #include "sol_attn.h"
@@ -133,6 +135,30 @@ size_t carve(const Shape& s, bool sol2, char* base, Work* w) {
   return off;
 }
 
+// The FP8 path's E4M3 operands and scales (after the buffers of carve()); bytes when base == nullptr.
+size_t carve_fp8(const Shape& s, char* base, Fp8Work* f) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes, 256);
+    return p;
+  };
+  const size_t tok = (size_t)s.B * s.N * s.H * kHeadDim, bh = (size_t)s.BH, nbp = (size_t)fp8_rows_padded(s);
+  Fp8Work t{};
+  t.q8 = reinterpret_cast<uint8_t*>(take(tok));
+  t.k8 = reinterpret_cast<uint8_t*>(take(tok));
+  t.v8 = reinterpret_cast<uint8_t*>(take(tok));
+  t.kbar8 = reinterpret_cast<uint8_t*>(take(bh * nbp * kHeadDim));
+  t.vbar8 = reinterpret_cast<uint8_t*>(take(bh * nbp * kHeadDim));
+  t.sq = reinterpret_cast<float*>(take(bh * s.Nb * 4));
+  t.sk = reinterpret_cast<float*>(take(bh * s.Nb * 4));
+  t.skbar = reinterpret_cast<float*>(take(bh * (nbp / 64) * 4));
+  t.sv = reinterpret_cast<float*>(take(bh * 4));
+  t.vmax = reinterpret_cast<unsigned int*>(take(bh * 4));
+  if (f) *f = t;
+  return off;
+}
+
 // Upper bound on the workspace of one device (0: none); lets callers cap the library's memory and
 // lets tests exercise the allocation-failure path without exhausting a GPU.
 size_t g_ws_limit = 0;
@@ -222,6 +248,30 @@ int encode_rows(CUtensorMap* m, const void* base, int rows, const Shape& s) {
 
 int encode_pooled(CUtensorMap* m, const void* base, const Shape& s) { return encode_rows(m, base, s.Nb, s); }
 
+// E4M3 BTHD bytes: 128 channels x 1 head x 64 tokens x 1 batch boxes (one 128-byte row per token).
+int encode_bthd8(CUtensorMap* m, const void* base, const Shape& s) {
+  const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)s.H, (cuuint64_t)s.N, (cuuint64_t)s.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)s.H * kHeadDim, (cuuint64_t)s.N * s.H * kHeadDim};
+  const cuuint32_t box[4] = {128, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOL_OK : fail(SOL_ERR_LAUNCH, "cuTensorMapEncodeTiled (E4M3 BTHD) failed: %d", (int)r);
+}
+
+// E4M3 [BH][rows][128] bytes, 128 x 128 x 1 boxes (compressed keys / values of the FP8 path).
+int encode_rows8(CUtensorMap* m, const void* base, int rows, const Shape& s) {
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)s.BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows * kHeadDim};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOL_OK : fail(SOL_ERR_LAUNCH, "cuTensorMapEncodeTiled (E4M3 rows) failed: %d", (int)r);
+}
+
 int check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "%s: %s", what, cudaGetErrorString(e));
@@ -283,13 +333,14 @@ int check_options(const sol_attn_options* o, int N, bool* diag, int* splits) {
 }
 
 int forward(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau, int sink_start,
-            int sink_tokens, const sol_attn_options* opts, void* stream, bool sol2) {
+            int sink_tokens, const sol_attn_options* opts, void* stream, bool sol2, bool fp8 = false) {
   int rc = validate(q, k, v, out, true, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
   bool diag;
   int splits;
   if ((rc = check_options(opts, N, &diag, &splits))) return rc;
   if (sol2 && splits > 1) return fail(SOL_ERR_OPTION, "kv_splits > 1 is available for Sol-Attn only");
+  if (fp8 && splits > 1) return fail(SOL_ERR_OPTION, "kv_splits > 1 is not available on the FP8 path");
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;
   int dev;
@@ -301,16 +352,27 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   const size_t rows_bh = (size_t)s.BH * s.QT * 128;
   const size_t part_o_bytes = splits > 1 ? (size_t)splits * rows_bh * 128 * 4 : 0;
   const size_t part_ml_bytes = splits > 1 ? (size_t)splits * rows_bh * 2 * 4 : 0;
-  if ((rc = ensure_workspace(*d, base + part_o_bytes + part_ml_bytes))) return rc;
+  const size_t fp8_bytes = fp8 ? carve_fp8(s, nullptr, nullptr) : 0;
+  if ((rc = ensure_workspace(*d, base + part_o_bytes + part_ml_bytes + fp8_bytes))) return rc;
   carve(s, sol2, static_cast<char*>(d->ws), &w);
+  Fp8Work f8{};
+  if (fp8) carve_fp8(s, static_cast<char*>(d->ws) + base + part_o_bytes + part_ml_bytes, &f8);
   float* part_o = splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(d->ws) + base) : nullptr;
   float* part_ml = splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(d->ws) + base + part_o_bytes) : nullptr;
   w.stats = d->stats;
 
   CUtensorMap maps[5];
-  if ((rc = encode_bthd(&maps[0], q, s)) || (rc = encode_bthd(&maps[1], k, s)) || (rc = encode_bthd(&maps[2], v, s)) ||
-      (rc = encode_pooled(&maps[3], w.kbar_h, s)) || (rc = encode_pooled(&maps[4], w.vbar_h, s)))
+  if (fp8) {
+    const int nbp = fp8_rows_padded(s);
+    if ((rc = encode_bthd8(&maps[0], f8.q8, s)) || (rc = encode_bthd8(&maps[1], f8.k8, s)) ||
+        (rc = encode_bthd8(&maps[2], f8.v8, s)) || (rc = encode_rows8(&maps[3], f8.kbar8, nbp, s)) ||
+        (rc = encode_rows8(&maps[4], f8.vbar8, nbp, s)))
+      return rc;
+  } else if ((rc = encode_bthd(&maps[0], q, s)) || (rc = encode_bthd(&maps[1], k, s)) ||
+             (rc = encode_bthd(&maps[2], v, s)) || (rc = encode_pooled(&maps[3], w.kbar_h, s)) ||
+             (rc = encode_pooled(&maps[4], w.vbar_h, s))) {
     return rc;
+  }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamWaitEvent(st, d->done, 0) != cudaSuccess) return fail(SOL_ERR_LAUNCH, "cudaStreamWaitEvent failed");
@@ -329,6 +391,11 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
     if (te != cudaSuccess) return fail(SOL_ERR_LAUNCH, "Sol-Attn2 tail launch: %s", cudaGetErrorString(te));
     launches += 3;
     if ((rc = check_launch("Sol-Attn2 tail kernels"))) return rc;
+  }
+  if (fp8) {
+    launch_quant_fp8(qh, kh, vh, s, w, f8, st);
+    launches += 3;
+    if ((rc = check_launch("FP8 quantisation kernels"))) return rc;
   }
   FwdParams p{};
   p.N = N;
@@ -358,7 +425,13 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
       return fail(SOL_ERR_LAUNCH, "timing event creation failed");
     cudaEventRecord(d->t0[slot], st);
   }
-  cudaError_t e = launch_attn_fwd(maps, p, s.BH * s.QT * splits, sol2, st);
+  cudaError_t e;
+  if (fp8) {
+    const Fp8Params fp{f8.sq, f8.sk, f8.skbar, f8.sv, fp8_rows_padded(s) / 64};
+    e = launch_attn_fwd_fp8(maps, p, fp, s.BH * s.QT, sol2, st);
+  } else {
+    e = launch_attn_fwd(maps, p, s.BH * s.QT * splits, sol2, st);
+  }
   if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "fused attention launch: %s", cudaGetErrorString(e));
   if (splits > 1) {
     launch_splitkv_combine(s, splits, part_o, part_ml, p.out, 0, N, st);
@@ -664,6 +737,28 @@ int sol_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, 
                            sink_tokens, opts, stream, false);
     if (rc) return rc;
   }
+  return SOL_OK;
+}
+
+int sol_attn_fwd_fp8(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                     int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream) {
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, opts, stream, false, true);
+}
+
+int sol_attn2_fwd_fp8(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                      int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream) {
+  return forward(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, opts, stream, true, true);
+}
+
+int sol_attn_expcast_host(const float* x, int n, float fs, float pivot, unsigned int* words) {
+  if (!x || !words) return fail(SOL_ERR_NULL, "x and words must be non-NULL");
+  if (n < 0 || n % 4) return fail(SOL_ERR_SHAPE, "n must be a non-negative multiple of 4 (got %d)", n);
+  if (!(fs > 0.f) || !std::isfinite(fs) || !std::isfinite(pivot) || pivot != std::floor(pivot))
+    return fail(SOL_ERR_OPTION, "fs must be positive and finite and pivot a finite integer");
+  const float c0 = kExpCastOffset - 8.0f * pivot;
+  for (int i = 0; i < n; i += 4)
+    words[i / 4] = pack_codes4(expcast_code_f32(x[i], 8.0f * fs, c0), expcast_code_f32(x[i + 1], 8.0f * fs, c0),
+                               expcast_code_f32(x[i + 2], 8.0f * fs, c0), expcast_code_f32(x[i + 3], 8.0f * fs, c0));
   return SOL_OK;
 }
 

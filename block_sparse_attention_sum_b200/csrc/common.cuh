@@ -96,4 +96,22 @@ void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bf
 cudaError_t launch_tail_tc(const void* maps, const Shape& s, const Work& w, int* status, cudaStream_t st);
 __host__ __device__ inline int tail_groups_padded(const Shape& s) { return (2 * s.Nb + 127) / 128 * 128; }
 
+// FP8 path (quant_fp8.cu, attn_fwd_fp8.cu): E4M3 operands and their scales.
+struct Fp8Work {
+  uint8_t* q8;            // [B][N][H][128]  E4M3 Q, one scale per (b, h, 64-token block)
+  uint8_t* k8;            // [B][N][H][128]  E4M3 K, same
+  uint8_t* v8;            // [B][N][H][128]  E4M3 V, one scale per (b, h)
+  uint8_t* kbar8;         // [BH][Nbp][128]  E4M3 compressed keys (block means), one scale per 64 rows
+  uint8_t* vbar8;         // [BH][Nbp][128]  E4M3 value means, the head's V scale
+  float* sq;              // [BH][Nb]
+  float* sk;              // [BH][Nb]
+  float* skbar;           // [BH][Nbp / 64]
+  float* sv;              // [BH]
+  unsigned int* vmax;     // [BH] max |V| of the head (float bits)
+};
+// Rows of the compressed-key arrays: Nb rounded up to whole 128-row surrogate chunks.
+__host__ __device__ inline int fp8_rows_padded(const Shape& s) { return (s.Nb + 127) / 128 * 128; }
+void launch_quant_fp8(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
+                      const Work& w, const Fp8Work& f, cudaStream_t st);
+
 }  // namespace sol

@@ -1,0 +1,130 @@
+// E4M3 tensor-core products and the ExpCast encoder of the FP8 forward.
+//
+// Sol-Attn2 draft, section "FP8 quantization and ExpCast": Q and K carry one E4M3 scale per 64-token
+// block, V one per head (s = max |X| / 448); QK and PV run on FP8 operands with FP32 accumulation;
+// ExpCast turns a base-2 score u relative to the shared pivot into the E4M3 probability byte
+// c(u) = clip_[0,120](RNE(8u + 55.65)), whose decoded value is about 2^u.
+#pragma once
+#include <cstdint>
+#include <cmath>
+
+namespace sol {
+
+// ExpCast constants: offset of the code line and the largest code (E4M3 0x78 = 2^8).
+constexpr float kExpCastOffset = 55.65f;
+constexpr int kExpCastMaxCode = 120;
+
+// The code of base-2 score x * fs against the integer pivot `pivot`, as the kernel computes it:
+// v = fma(x, 8 fs, 55.65 - 8 pivot) (one rounding), clamped below at 0, rounded to the nearest
+// integer (ties to even) by adding 1.5 * 2^23, whose unit in the last place is 1: the rounded value
+// is then the low byte of the sum's bit pattern.  The clip at 120 is not applied: the pivot rule
+// keeps x * fs <= pivot + 8, so v <= 119.65 up to the FP32 rounding of the products.  A masked
+// score (x = -inf) gives code 0, the E4M3 encoding of +0.
+__host__ __device__ __forceinline__ uint32_t expcast_code_f32(float x, float f8, float c) {
+  float v = fmaf(x, f8, c);
+  v = fmaxf(v, 0.0f);
+  const float r = v + 12582912.0f;
+  uint32_t bits;
+#ifdef __CUDA_ARCH__
+  bits = __float_as_uint(r);
+#else
+  __builtin_memcpy(&bits, &r, 4);
+#endif
+  return bits & 0xffu;
+}
+
+// Four codes in one 32-bit word, the first key in the low byte: the layout of an E4M3 A operand in
+// tensor memory (one row per lane, four consecutive K elements per 32-bit column).
+__host__ __device__ __forceinline__ uint32_t pack_codes4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3) {
+  return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+}
+
+// 2^k for an integer-valued float k (exact; 0 below the normal range, k = -inf included).
+__host__ __device__ __forceinline__ float pow2i(float k) {
+  if (!(k >= -126.0f)) return 0.0f;
+  const int e = (int)k + 127;
+  const uint32_t bits = (uint32_t)(e > 254 ? 254 : e) << 23;
+  float r;
+#ifdef __CUDA_ARCH__
+  r = __uint_as_float(bits);
+#else
+  __builtin_memcpy(&r, &bits, 4);
+#endif
+  return r;
+}
+
+// Pivot rule of the online softmax: the pivot is an integer (base 2) and moves only when the running
+// maximum exceeds it by more than 8, to ceil(max) - 8, so that every coded score satisfies u <= 8.
+// Returns the new pivot; *alpha = 2^(old - new) rescales what was accumulated against the old one
+// (0 when there was none).
+__host__ __device__ __forceinline__ float pivot_update(float pivot, float mx, float* alpha, bool* moved) {
+  if (mx > pivot + 8.0f) {
+    const float np = ceilf(mx) - 8.0f;
+    *alpha = pow2i(pivot - np);
+    *moved = true;
+    return np;
+  }
+  *alpha = 1.0f;
+  *moved = false;
+  return pivot;
+}
+
+#ifdef __CUDACC__
+// Instruction descriptor, kind::f8f6f4: E4M3 A and B (format 0), FP32 accumulator, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem], E4M3 operands, K = 32 per instruction; one thread issues.
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]: A (M x K, E4M3) from tensor memory, one row per lane, four K
+// elements per 32-bit column (lowest K index in the low byte).
+__device__ __forceinline__ void umma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 bit, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// One column per thread (32 lanes x 32 bit).
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return r;
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
+
+// Two FP32 values to two E4M3 bytes (round to nearest even, saturating at +-448), lo in the low byte.
+__device__ __forceinline__ uint32_t to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+#endif  // __CUDACC__
+
+}  // namespace sol

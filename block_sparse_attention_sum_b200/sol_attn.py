@@ -37,6 +37,9 @@ EXPORTS = [
     "sol_attn_dense_rows",
     "sol_attn_set_workspace_limit",
     "sol_attn_selftest_wait_timeout",
+    "sol_attn_fwd_fp8",
+    "sol_attn2_fwd_fp8",
+    "sol_attn_expcast_host",
 ]
 
 STATUS = {
@@ -138,6 +141,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_set_workspace_limit.restype = None
     lib.sol_attn_selftest_wait_timeout.argtypes = [vp]
     lib.sol_attn_selftest_wait_timeout.restype = i
+    lib.sol_attn_fwd_fp8.argtypes = ex_args
+    lib.sol_attn_fwd_fp8.restype = i
+    lib.sol_attn2_fwd_fp8.argtypes = ex_args
+    lib.sol_attn2_fwd_fp8.restype = i
+    lib.sol_attn_expcast_host.argtypes = [ctypes.POINTER(ctypes.c_float), i, f, f, ctypes.POINTER(ctypes.c_uint)]
+    lib.sol_attn_expcast_host.restype = i
     _lib = lib
     return lib
 
@@ -197,6 +206,48 @@ def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stre
                   extra_sinks=()):
     """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
     return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks)
+
+
+def _fwd_fp8(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks):
+    B, N, H = _check_qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device != q.device:
+        raise ValueError("out must be a contiguous BF16 tensor shaped like q")
+    opts = _options(thresh_type, extra_sinks)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = getattr(lib, fn_name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, float(tau),
+                                   int(sink_start), int(sink_tokens), ctypes.byref(opts), _stream_handle(stream))
+    _check(rc)
+    return out
+
+
+def sol_attn_fwd_fp8(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
+                     extra_sinks=()):
+    """FP8 (E4M3) + ExpCast Sol-Attn forward: BF16 inputs and output, E4M3 attention products."""
+    return _fwd_fp8("sol_attn_fwd_fp8", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks)
+
+
+def sol_attn2_fwd_fp8(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
+                      extra_sinks=()):
+    """FP8 (E4M3) + ExpCast Sol-Attn2 forward (complementary tail as in the BF16 path)."""
+    return _fwd_fp8("sol_attn2_fwd_fp8", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type,
+                    extra_sinks)
+
+
+def expcast_host(x, fs: float, pivot: float):
+    """The FP8 kernels' ExpCast encoder evaluated on the host: uint8 codes of x * fs - pivot (x a
+    sequence of floats, length a multiple of 4), unpacked from the library's 32-bit words."""
+    import numpy as np
+
+    xs = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    words = np.zeros(xs.size // 4, dtype=np.uint32)
+    lib = load_library()
+    rc = lib.sol_attn_expcast_host(xs.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), int(xs.size), float(fs),
+                                   float(pivot), words.ctypes.data_as(ctypes.POINTER(ctypes.c_uint)))
+    _check(rc)
+    return words.view(np.uint8).copy()
 
 
 def sol_attn_fwd_varlen(q, k, v, cu_seqlens, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None,

@@ -256,6 +256,46 @@ void sol_attn_set_workspace_limit(size_t bytes);
  */
 int sol_attn_selftest_wait_timeout(void* stream);
 
+/*
+ * FP8 (E4M3) + ExpCast forward ("Sol-Attn2" draft, section "FP8 quantization and ExpCast").  Same
+ * arguments, routing and exact sets as sol_attn_fwd_ex / sol_attn2_fwd_ex (BF16 inputs and output;
+ * the routing is computed from the BF16 inputs exactly as there).  The attention products then run
+ * on E4M3 operands with FP32 accumulation:
+ *   - Q and K are quantised with one scale per (b, h, 64-token block), V with one per (b, h):
+ *     s = max |X| / 448 (1 for an all-zero block), X8 = E4M3(X / s), round to nearest even,
+ *     saturating.  sol_attn_fwd_fp8's surrogate keys Kbar_j take one scale per 64 consecutive key
+ *     blocks of a (b, h), its value means Vbar_j = Vhat_j / n_j the head's V scale; a surrogate
+ *     block's logit is q8 . Kbar8_j / sqrt(128) + ln n_j.
+ *   - Every softmax weight is an ExpCast byte: with u the base-2 score minus the row's pivot,
+ *     c(u) = clip_[0,120](RNE(8u + 55.65)), weight decode_E4M3(c) ~= 2^u (within 7.5 %).  The pivot is
+ *     an integer that moves only when the running maximum exceeds it by more than 8, to
+ *     ceil(max) - 8.  The same decoded weights enter the P V product and the denominator.
+ *   - sol_attn2_fwd_fp8: the exact branch as above; the complementary tail (Z_a, mu_a, nu_a) as in
+ *     sol_attn2_fwd from the BF16 inputs, with delta_i taken from the dequantised query, merged
+ *     into the denominator with its exact exponential.
+ * Results differ from the BF16 entry points by the E4M3 and ExpCast roundings (about 5 % relative
+ * L2 on unit-variance inputs).  kv_splits > 1 returns SOL_ERR_OPTION.  The workspace grows by
+ * 3 * B*N*H*128 bytes (E4M3 copies of Q, K, V) plus the compressed operands and scales.
+ * Kernel timing (sol_attn_set_kernel_timing) covers the fused kernel only; the quantisation
+ * kernels run before it, after the routing.
+ */
+int sol_attn_fwd_fp8(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                     int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream);
+int sol_attn2_fwd_fp8(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                      int sink_start, int sink_tokens, const sol_attn_options* opts, void* stream);
+
+/*
+ * Host evaluation of the FP8 kernels' ExpCast encoder (the same inline function the softmax runs;
+ * for checking it against a reference without a GPU).  For n scores x (HOST floats, n a multiple
+ * of 4), base-2 multiplier fs > 0 and integer pivot: code_i = the E4M3 byte of
+ * u_i = x_i * fs - pivot computed as max(fma(x_i, 8 fs, 55.65 - 8 pivot), 0) rounded to the nearest
+ * integer (ties to even); words[i / 4] holds codes i .. i + 3, the first in the low byte (the
+ * layout of a P operand column in tensor memory).  The clip at 120 is the caller's invariant
+ * u <= 8 (the kernels' pivot rule keeps it).  Returns SOL_ERR_NULL, SOL_ERR_SHAPE (n) or
+ * SOL_ERR_OPTION (fs, pivot) without writing.
+ */
+int sol_attn_expcast_host(const float* x, int n, float fs, float pivot, unsigned int* words);
+
 #ifdef __cplusplus
 }
 #endif

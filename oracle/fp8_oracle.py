@@ -35,6 +35,12 @@ R19 ExpCast gives every weight of the shared softmax, exact tokens and surrogate
     (u <= 8, the largest weight coded 112..120), the same range an online pivot moved only when the
     running maximum exceeds it by more than 8 keeps.
 R20 An all-zero quantisation block keeps scale 1 and zero codes.
+R21 Sol-Attn2 under FP8: the exact branch as above (E4M3 operands, ExpCast weights against the
+    integer pivot ceil(max exact score / ln 2) - 8); the complementary tail's Z_a, mu_a, nu_a are
+    those of the BF16 path (computed from the original inputs: the tail is not a product of the
+    shared softmax); delta_i takes the dequantised query s_Q Q8_i, and Zhat_i enters the shared
+    denominator with its exact exponential relative to the same pivot (one term per row, not a
+    probability byte of a PV product).
 """
 from __future__ import annotations
 
@@ -149,4 +155,55 @@ def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0
             for i in (range(Nb) if qblocks is None else qblocks):
                 lo, hi = orc.block_range(i, N)
                 out[b, lo:hi, h] = sol_attn_fp8_rows(q8[lo:hi], k8, v8, r["mask"][i], kbar8, vbar8, r["counts"])
+    return dict(out=out, mask=masks)
+
+
+def sol_attn2_fp8_rows(q8_rows, row0, k8_bh, v8_bh, mask_row, counts, kg, vg, qbar_anchor):
+    """Outputs of the query rows [row0, row0 + len) of one query block under FP8 Sol-Attn2 (R21)."""
+    N = k8_bh.shape[0]
+    ex = np.nonzero(mask_row)[0]
+    un = np.nonzero(~mask_row)[0]
+    tok = np.concatenate([np.arange(*orc.block_range(j, N)) for j in ex]) if len(ex) else np.zeros(0, np.int64)
+    z = orc.SCALE * (q8_rows @ k8_bh[tok].T)
+    t_counts = counts[un].reshape(-1)
+    t_k = kg[un].reshape(-1, orc.HEAD_DIM)
+    t_v = vg[un].reshape(-1, orc.HEAD_DIM)
+    keep = t_counts > 0
+    t_counts, t_k, t_v = t_counts[keep], t_k[keep], t_v[keep]
+    out = np.empty_like(q8_rows)
+    for r in range(q8_rows.shape[0]):
+        a = (row0 + r) // orc.ANCHOR
+        logZ, mu_a, nu_a = orc.anchor_tail(qbar_anchor[a], t_counts, t_k, t_v)
+        zr = z[r]
+        pivot = (np.ceil(zr.max() / math.log(2.0)) - 8.0) if zr.size else 0.0
+        pz = expcast(zr / math.log(2.0) - pivot)
+        if np.isfinite(logZ):
+            delta = orc.SCALE * ((q8_rows[r] - qbar_anchor[a]) @ mu_a)
+            zt = math.exp(logZ + delta - pivot * math.log(2.0))
+        else:
+            zt = 0.0
+        out[r] = (pz @ v8_bh[tok] + zt * nu_a) / (pz.sum() + zt)
+    return out
+
+
+def sol_attn2_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None):
+    """FP8 + ExpCast Sol-Attn2 forward (R21).  Same return convention as :func:`sol_attn_fp8`."""
+    B, N, H, _ = q.shape
+    Nb = orc.num_blocks(N)
+    sink = orc.sink_block_flags(N, sink_start, sink_tokens)
+    out = np.full((B, N, H, orc.HEAD_DIM), np.nan)
+    masks = np.zeros((B, H, Nb, Nb), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            q_bh, k_bh, v_bh = orc.head_slice(q, b, h), orc.head_slice(k, b, h), orc.head_slice(v, b, h)
+            r = orc._routing_for_head(q_bh, k_bh, tau, sink)
+            masks[b, h] = r["mask"]
+            counts, kg, vg = orc.key_groups(k_bh, v_bh, q_bh.mean(axis=0))
+            qbar_anchor = orc.block_means(q_bh, orc.ANCHOR)
+            q8, k8 = quantize_blocks(q_bh), quantize_blocks(k_bh)
+            v8 = quantize(v_bh)[0]
+            for i in (range(Nb) if qblocks is None else qblocks):
+                lo, hi = orc.block_range(i, N)
+                out[b, lo:hi, h] = sol_attn2_fp8_rows(q8[lo:hi], lo, k8, v8, r["mask"][i], counts, kg, vg,
+                                                      qbar_anchor)
     return dict(out=out, mask=masks)

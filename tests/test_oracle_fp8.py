@@ -104,3 +104,36 @@ def test_fp8_forward_error_is_that_of_its_roundings():
     b = orc.sol_attn(q, k, v, tau=1.0)["out"]
     rel = np.linalg.norm(a - b) / np.linalg.norm(b)
     assert 0.005 < rel < 0.1, rel
+
+
+def test_fp8_sol2_reduces_to_the_bf16_sol2_without_rounding(monkeypatch):
+    monkeypatch.setattr(f8, "expcast", lambda u: 2.0 ** np.asarray(u))
+    monkeypatch.setattr(f8, "e4m3_round", lambda x: np.asarray(x, dtype=np.float64))
+    g = np.random.default_rng(7)
+    q, k, v = (g.standard_normal((1, 600, 2, 128)) for _ in range(3))
+    a = f8.sol_attn2_fp8(q, k, v, tau=0.5, sink_start=0, sink_tokens=64)["out"]
+    b = orc.sol_attn2(q, k, v, tau=0.5, sink_start=0, sink_tokens=64)["out"]
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_fp8_sol2_with_zero_queries_averages_the_values():
+    # q = 0: exact scores 0 give the ExpCast weight 2^8 (u = 8 against the pivot -8); the tail of an
+    # anchor has Z_a = its token count, nu_a = the mean of its values and delta = 0, so with V on the
+    # E4M3 grid the output is the mean of V over all tokens.
+    N, H = 640, 1
+    g = np.random.default_rng(8)
+    q = np.zeros((1, N, H, 128))
+    k = g.standard_normal((1, N, H, 128))
+    v = g.choice([-1.0, -0.5, 0.0, 0.5, 1.0], size=(1, N, H, 128))
+    v[0, 0, :, 0] = 1.0
+    out = f8.sol_attn2_fp8(q, k, v, tau=1.0)["out"]
+    np.testing.assert_allclose(out[0], np.broadcast_to(v[0].mean(axis=0), (N, H, 128)), rtol=0, atol=1e-12)
+
+
+def test_fp8_sol2_error_is_that_of_its_roundings():
+    g = np.random.default_rng(10)
+    q, k, v = (g.standard_normal((1, 640, 1, 128)) for _ in range(3))
+    a = f8.sol_attn2_fp8(q, k, v, tau=1.0)["out"]
+    b = orc.sol_attn2(q, k, v, tau=1.0)["out"]
+    rel = np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert 0.005 < rel < 0.1, rel

@@ -156,6 +156,28 @@ def _surrogate_sums_quantised(Kbar, Vhat, counts, v_scale):
 _orig_surrogate = f8.surrogate_operands_fp8
 
 
+def _sol2_fp8_tail_without_pivot(q8_rows, row0, k8_bh, v8_bh, mask_row, counts, kg, vg, qbar_anchor):
+    # the tail mass added without the pivot's factor 2^-pivot
+    import math as _m
+    from oracle import sol_attn_oracle as _orc
+    N = k8_bh.shape[0]
+    ex = np.nonzero(mask_row)[0]
+    un = np.nonzero(~mask_row)[0]
+    tok = np.concatenate([np.arange(*_orc.block_range(j, N)) for j in ex])
+    z = _orc.SCALE * (q8_rows @ k8_bh[tok].T)
+    tc, tk, tv = counts[un].reshape(-1), kg[un].reshape(-1, 128), vg[un].reshape(-1, 128)
+    keep = tc > 0
+    out = np.empty_like(q8_rows)
+    for r in range(q8_rows.shape[0]):
+        a = (row0 + r) // _orc.ANCHOR
+        logZ, mu_a, nu_a = _orc.anchor_tail(qbar_anchor[a], tc[keep], tk[keep], tv[keep])
+        pivot = np.ceil(z[r].max() / _m.log(2.0)) - 8.0
+        pz = f8.expcast(z[r] / _m.log(2.0) - pivot)
+        zt = _m.exp(logZ + _orc.SCALE * ((q8_rows[r] - qbar_anchor[a]) @ mu_a)) if np.isfinite(logZ) else 0.0
+        out[r] = (pz @ v8_bh[tok] + zt * nu_a) / (pz.sum() + zt)
+    return out
+
+
 FP8_CASES = [
     ("e4m3_decode", _decode_bias_8, fp8pins.test_e4m3_decode_matches_torch),
     ("expcast_code", lambda u: np.round(8.0 * np.asarray(u) + f8.EXPCAST_OFFSET).astype(np.int64),
@@ -169,6 +191,7 @@ FP8_CASES = [
      fp8pins.test_surrogate_operands_are_quantised_like_keys_and_values),
     ("surrogate_operands_fp8", _surrogate_sums_quantised,
      fp8pins.test_fp8_forward_with_zero_queries_averages_the_values),
+    ("sol_attn2_fp8_rows", _sol2_fp8_tail_without_pivot, fp8pins.test_fp8_sol2_with_zero_queries_averages_the_values),
 ]
 
 
