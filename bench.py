@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--kv-splits", type=int, default=1,
                     help="split-KV shares per 128-row query tile (Sol-Attn only; 1 = off)")
+    ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"],
+                    help="attention products in BF16 (default) or E4M3 with ExpCast weights (sol_attn*_fwd_fp8)")
     return ap.parse_args()
 
 
@@ -275,7 +277,13 @@ def main():
     q, k, v = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
     out = torch.empty_like(q)
     tau = w.resolved_tau()
-    fn = sa.sol_attn_fwd if w.entry == "sol_attn" else sa.sol_attn2_fwd
+    fp8 = args.precision == "fp8"
+    if fp8 and args.kv_splits != 1:
+        raise SystemExit("--kv-splits is not available with --precision fp8")
+    if fp8:
+        fn = sa.sol_attn_fwd_fp8 if w.entry == "sol_attn" else sa.sol_attn2_fwd_fp8
+    else:
+        fn = sa.sol_attn_fwd if w.entry == "sol_attn" else sa.sol_attn2_fwd
     stream = torch.cuda.current_stream()
 
     extra = {"kv_splits": args.kv_splits} if args.kv_splits != 1 else {}
@@ -350,23 +358,29 @@ def main():
                "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": e2e_steps}
 
     peaks = load_peaks()
-    peak_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    peak_burst = float(peaks["bf16_tflops"])
+    # E4M3 products: the measured BF16 peak times the nominal dense FP8 / BF16 ratio (4.5 / 2.25)
+    ratio = 2.0 if fp8 else 1.0
+    peak_sust = ratio * float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    peak_burst = ratio * float(peaks["bf16_tflops"])
     achieved = flops_step / (kernel_ms * 1e-3) / 1e12
+    kname = ("attn_fwd_fp8_kernel" if fp8 else "attn_fwd_kernel") + ("<false>" if w.entry == "sol_attn" else "<true>")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sust, "unit": "TFLOP/s",
-                "frac": achieved / peak_sust, "traffic": measured_traffic(w.name),
-                "kernel": "attn_fwd_kernel<false> (fused routing + attention)",
-                "kernel_ms": kernel_ms, "peak_kind": f"bf16 dense sustained ({peaks['source']})",
+                "frac": achieved / peak_sust, "traffic": None if fp8 else measured_traffic(w.name),
+                "kernel": kname + " (fused attention)",
+                "kernel_ms": kernel_ms,
+                "peak_kind": (f"e4m3 dense sustained = 2 x measured bf16 ({peaks['source']})" if fp8 else
+                              f"bf16 dense sustained ({peaks['source']})"),
                 "frac_of_burst": achieved / peak_burst}
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
             "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d=128 GRF t-major {w.grid.T}x{w.grid.Y}x{w.grid.X}"
                                    if w.grid else w.name,
                        "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "tau": tau,
                        "target_sparsity": w.target_sparsity, "realised_sparsity": sp,
                        "union_tile_useful_fraction": union_frac, "kv_splits": args.kv_splits,
+                       "precision": args.precision,
                        "parallelism": f"independent replicas x{world} (head/batch sharding, no exchange)",
                        "l2": "inputs 1.6 GB per rank > 126 MB L2; no flush"},
             "frac_of_peak": value / world / peak_burst, "frac_of_sustained_peak": value / world / peak_sust,
