@@ -307,11 +307,15 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   return check_launch("routing kernels");
 }
 
-// Validates the options against the sequence length; sets *diag and *splits.
-int check_options(const sol_attn_options* o, int N, bool* diag, int* splits) {
+// Validates the options against the sequence length; sets *diag, *splits and *fp8.
+int check_options(const sol_attn_options* o, int N, bool* diag, int* splits, bool* fp8) {
   *diag = false;
   *splits = 1;
+  *fp8 = false;
   if (!o) return SOL_OK;
+  if (o->precision != SOL_PRECISION_BF16 && o->precision != SOL_PRECISION_FP8)
+    return fail(SOL_ERR_OPTION, "unknown precision %d", o->precision);
+  *fp8 = o->precision == SOL_PRECISION_FP8;
   if (o->kv_splits < 0 || o->kv_splits > SOL_MAX_KV_SPLITS)
     return fail(SOL_ERR_OPTION, "kv_splits must be in [0, %d]", SOL_MAX_KV_SPLITS);
   *splits = o->kv_splits > 1 ? o->kv_splits : 1;
@@ -336,9 +340,10 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
             int sink_tokens, const sol_attn_options* opts, void* stream, bool sol2, bool fp8 = false) {
   int rc = validate(q, k, v, out, true, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
-  bool diag;
+  bool diag, opt_fp8;
   int splits;
-  if ((rc = check_options(opts, N, &diag, &splits))) return rc;
+  if ((rc = check_options(opts, N, &diag, &splits, &opt_fp8))) return rc;
+  fp8 = fp8 || opt_fp8;
   if (sol2 && splits > 1) return fail(SOL_ERR_OPTION, "kv_splits > 1 is available for Sol-Attn only");
   if (fp8 && splits > 1) return fail(SOL_ERR_OPTION, "kv_splits > 1 is not available on the FP8 path");
   std::lock_guard<std::mutex> lock(g_mu);
@@ -586,7 +591,8 @@ int sol_attn_debug_route_ex(const void* q, const void* k, int B, int N, int H, f
   if (rc) return rc;
   bool diag;
   int splits;
-  if ((rc = check_options(opts, N, &diag, &splits))) return rc;
+  bool fp8_unused;
+  if ((rc = check_options(opts, N, &diag, &splits, &fp8_unused))) return rc;
   if (!mask) return fail(SOL_ERR_NULL, "mask must be non-NULL");
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* d;

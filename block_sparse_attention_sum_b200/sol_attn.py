@@ -49,6 +49,7 @@ STATUS = {
 }
 
 THRESH_TYPES = {"exact": 0, "diag": 1}
+PRECISIONS = {"bf16": 0, "fp8": 1}
 MAX_EXTRA_SINKS = 4
 MAX_KV_SPLITS = 8
 
@@ -58,14 +59,16 @@ class Options(ctypes.Structure):
 
     _fields_ = [("thresh_type", ctypes.c_int), ("n_extra_sinks", ctypes.c_int),
                 ("extra_sink_start", ctypes.c_int * MAX_EXTRA_SINKS), ("extra_sink_tokens", ctypes.c_int * MAX_EXTRA_SINKS),
-                ("kv_splits", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
+                ("kv_splits", ctypes.c_int), ("precision", ctypes.c_int), ("reserved", ctypes.c_int * 4)]
 
 
-def _options(thresh_type: str, extra_sinks=(), kv_splits: int = 1):
+def _options(thresh_type: str, extra_sinks=(), kv_splits: int = 1, precision: str = "bf16"):
     """extra_sinks: up to MAX_EXTRA_SINKS (start, tokens) token ranges made exact for every query;
-    kv_splits: split-KV shares per query tile (1 = off)."""
+    kv_splits: split-KV shares per query tile (1 = off); precision: "bf16" or "fp8" (E4M3 + ExpCast)."""
     if thresh_type not in THRESH_TYPES:
         raise ValueError(f"thresh_type must be one of {sorted(THRESH_TYPES)}")
+    if precision not in PRECISIONS:
+        raise ValueError(f"precision must be one of {sorted(PRECISIONS)}")
     extra_sinks = list(extra_sinks)
     if len(extra_sinks) > MAX_EXTRA_SINKS:
         raise ValueError(f"at most {MAX_EXTRA_SINKS} extra sink ranges")
@@ -73,6 +76,7 @@ def _options(thresh_type: str, extra_sinks=(), kv_splits: int = 1):
     o.thresh_type = THRESH_TYPES[thresh_type]
     o.n_extra_sinks = len(extra_sinks)
     o.kv_splits = int(kv_splits)
+    o.precision = PRECISIONS[precision]
     for e, (start, tokens) in enumerate(extra_sinks):
         o.extra_sink_start[e] = int(start)
         o.extra_sink_tokens[e] = int(tokens)
@@ -176,7 +180,7 @@ def _check_qkv(q, k, v=None):
 
 
 def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type="exact", extra_sinks=(),
-         kv_splits=1):
+         kv_splits=1, precision="bf16"):
     B, N, H = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
@@ -186,8 +190,8 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
     args = [q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, float(tau), int(sink_start),
             int(sink_tokens)]
     with torch.cuda.device(q.device):
-        if thresh_type != "exact" or extra_sinks or kv_splits != 1:
-            opts = _options(thresh_type, extra_sinks, kv_splits)
+        if thresh_type != "exact" or extra_sinks or kv_splits != 1 or precision != "bf16":
+            opts = _options(thresh_type, extra_sinks, kv_splits, precision)
             rc = getattr(lib, fn_name + "_ex")(*args, ctypes.byref(opts), _stream_handle(stream))
         else:
             rc = getattr(lib, fn_name)(*args, _stream_handle(stream))
@@ -196,16 +200,17 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
 
 
 def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
-                 extra_sinks=(), kv_splits=1):
+                 extra_sinks=(), kv_splits=1, precision="bf16"):
     """Sol-Attn forward through the C ABI; returns ``out`` (BF16 [B, N, H, 128])."""
     return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks,
-                kv_splits)
+                kv_splits, precision)
 
 
 def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
-                  extra_sinks=()):
+                  extra_sinks=(), precision="bf16"):
     """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
-    return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks)
+    return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks,
+                precision=precision)
 
 
 def _fwd_fp8(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks):
@@ -251,7 +256,7 @@ def expcast_host(x, fs: float, pivot: float):
 
 
 def sol_attn_fwd_varlen(q, k, v, cu_seqlens, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None,
-                        thresh_type="exact", extra_sinks=(), kv_splits=1):
+                        thresh_type="exact", extra_sinks=(), kv_splits=1, precision="bf16"):
     """Packed variable-length batch: q, k, v BF16 [total_tokens, H, 128]; sequence s is the tokens
     cu_seqlens[s] .. cu_seqlens[s + 1] - 1 (a host list of offsets starting at 0)."""
     for t in (q, k, v):
@@ -264,7 +269,7 @@ def sol_attn_fwd_varlen(q, k, v, cu_seqlens, tau=1.0, sink_start=-1, sink_tokens
     if cu[-1] > q.shape[0]:
         raise ValueError("cu_seqlens exceeds the packed token count")
     arr = (ctypes.c_int * len(cu))(*cu)
-    opts = _options(thresh_type, extra_sinks, kv_splits)
+    opts = _options(thresh_type, extra_sinks, kv_splits, precision)
     lib = load_library()
     with torch.cuda.device(q.device):
         rc = lib.sol_attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), arr, len(cu) - 1,

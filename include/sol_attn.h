@@ -67,6 +67,12 @@ typedef enum {
 #define SOL_MAX_EXTRA_SINKS 4
 #define SOL_MAX_KV_SPLITS 8
 
+/* Arithmetic of the attention products (sol_attn_options.precision). */
+typedef enum {
+  SOL_PRECISION_BF16 = 0, /* BF16 operands, FP32 accumulation and exponentials (the default) */
+  SOL_PRECISION_FP8 = 1   /* E4M3 operands and ExpCast weights, as sol_attn_fwd_fp8 / sol_attn2_fwd_fp8 */
+} sol_precision;
+
 /*
  * Options of the _ex entry points.  A NULL pointer means all defaults (an all-zero struct is the
  * default too); reserved fields must be 0.
@@ -85,6 +91,10 @@ typedef enum {
  *                      unsplit call up to FP32 rounding.  Raises parallelism when there are few
  *                      query tiles; the workspace grows by kv_splits * B*H*ceil(N/128)*128 * 520
  *                      bytes.  Sol-Attn only: sol_attn2_fwd_ex rejects kv_splits > 1.
+ *   precision          sol_precision.  SOL_PRECISION_FP8 makes sol_attn_fwd_ex, sol_attn2_fwd_ex and
+ *                      sol_attn_fwd_varlen run the FP8 path of sol_attn_fwd_fp8 / sol_attn2_fwd_fp8;
+ *                      it cannot be combined with kv_splits > 1.  The routing (and so
+ *                      sol_attn_debug_route_ex) is the same for both.
  */
 typedef struct {
   int thresh_type;
@@ -92,7 +102,8 @@ typedef struct {
   int extra_sink_start[SOL_MAX_EXTRA_SINKS];
   int extra_sink_tokens[SOL_MAX_EXTRA_SINKS];
   int kv_splits;
-  int reserved[5];
+  int precision;
+  int reserved[4];
 } sol_attn_options;
 
 /*

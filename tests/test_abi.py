@@ -83,6 +83,13 @@ def test_invalid_options_are_rejected_on_the_host(lib):
     assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
     opts = sa._options("exact", kv_splits=-1)
     assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa.Options()
+    opts.precision = 7                              # unknown precision
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa._options("exact", kv_splits=2, precision="fp8")   # no split-KV on the FP8 path
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    with pytest.raises(ValueError):
+        sa._options("exact", precision="fp16")
 
 
 def test_options_struct_matches_the_header():
@@ -90,6 +97,8 @@ def test_options_struct_matches_the_header():
     assert "#define SOL_MAX_EXTRA_SINKS 4" in text and sa.MAX_EXTRA_SINKS == 4
     assert "#define SOL_MAX_KV_SPLITS 8" in text and sa.MAX_KV_SPLITS == 8
     assert ctypes.sizeof(sa.Options) == 16 * 4
+    assert "SOL_PRECISION_BF16 = 0" in text and "SOL_PRECISION_FP8 = 1" in text and sa.PRECISIONS == {"bf16": 0, "fp8": 1}
+    assert sa.Options.precision.offset == 11 * 4 and sa.Options.reserved.offset == 12 * 4
 
 
 def test_dense_rows_host_validation(lib):

@@ -150,3 +150,19 @@ def test_fp8_is_close_to_bf16_and_deterministic():
     assert torch.equal(a, b)
     rel = float((a.float() - c.float()).norm() / c.float().norm())
     assert 0.005 < rel < 0.1, rel
+
+
+def test_fp8_precision_option_and_varlen_match_the_fp8_entry_points():
+    q, k, v = (t.cuda() for t in iid_qkv(1, 1000, 2, seed=23))
+    a = sa.sol_attn_fwd_fp8(q, k, v, 1.0)
+    b = sa.sol_attn_fwd(q, k, v, 1.0, precision="fp8")
+    c = sa.sol_attn2_fwd_fp8(q, k, v, 1.0)
+    d = sa.sol_attn2_fwd(q, k, v, 1.0, precision="fp8")
+    cu = [0, 300, 300, 1000]
+    pv = sa.sol_attn_fwd_varlen(q[0], k[0], v[0], cu, 1.0, precision="fp8")
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(c, d)
+    for s0, s1 in zip(cu[:-1], cu[1:]):
+        if s1 > s0:
+            one = sa.sol_attn_fwd_fp8(q[:, s0:s1].contiguous(), k[:, s0:s1].contiguous(), v[:, s0:s1].contiguous(), 1.0)
+            assert torch.equal(pv[s0:s1], one[0])
