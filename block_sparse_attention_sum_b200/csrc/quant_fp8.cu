@@ -55,11 +55,18 @@ __device__ __forceinline__ void load_rows_bf16(const __nv_bfloat16* x, const Sha
   *amax = m;
 }
 
-// Eight values divided by the scale, as four E4M3 pairs in one 8-byte word.
-__device__ __forceinline__ uint2 codes8(const float (&v)[8], float sc) {
+// X / s with s = m / 448, evaluated as (x * 448) / m: for a BF16 x the product is exact and the
+// quotient is correctly rounded, so a value that lies exactly halfway between two E4M3 numbers
+// (frequent: x and m share most of their few mantissa bits) stays exactly halfway and rounds to
+// even, as the definition asks; x / fl(m / 448) can land just off the midpoint and round the
+// other way.  m > 0.
+__device__ __forceinline__ float scaled448(float x, float m) { return (x * 448.0f) / m; }
+
+// Eight values of a block with maximum |X| = m > 0, as four E4M3 pairs in one 8-byte word.
+__device__ __forceinline__ uint2 codes8(const float (&v)[8], float m) {
   uint32_t w[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) w[e] = to_e4m3x2(v[2 * e] / sc, v[2 * e + 1] / sc);
+  for (int e = 0; e < 4; ++e) w[e] = to_e4m3x2(scaled448(v[2 * e], m), scaled448(v[2 * e + 1], m));
   return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
@@ -91,7 +98,7 @@ __global__ void __launch_bounds__(256) quant_qk_kernel(const __nv_bfloat16* __re
     const int row = rg + 16 * r;
     if (row < n)
       *reinterpret_cast<uint2*>(x8 + (((size_t)b * s.N + t0 + row) * s.H + h) * kHeadDim + 8 * c16) =
-          codes8(vals[r], sc);
+          m > 0.f ? codes8(vals[r], m) : make_uint2(0u, 0u);
   }
 }
 
@@ -114,7 +121,7 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const __nv_bfloat16* __res
     const int row = rg + 16 * r;
     if (row < n)
       *reinterpret_cast<uint2*>(v8 + (((size_t)b * s.N + t0 + row) * s.H + h) * kHeadDim + 8 * c16) =
-          codes8(vals[r], sc);
+          m > 0.f ? codes8(vals[r], m) : make_uint2(0u, 0u);
   }
   // column sums: rows beyond n were loaded as zeros
 #pragma unroll
@@ -128,7 +135,7 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const __nv_bfloat16* __res
       a1 += colsum[g][2 * tid + 1];
     }
     const float inv_n = 1.0f / (float)n;
-    const uint32_t w = to_e4m3x2((a0 * inv_n) / sc, (a1 * inv_n) / sc);
+    const uint32_t w = m > 0.f ? to_e4m3x2(scaled448(a0 * inv_n, m), scaled448(a1 * inv_n, m)) : 0u;
     *reinterpret_cast<uint16_t*>(vbar8 + ((size_t)bh * Nbp + j) * kHeadDim + 2 * tid) = (uint16_t)w;
   }
 }
@@ -164,7 +171,7 @@ __global__ void __launch_bounds__(256) quant_kbar_kernel(const float* __restrict
   for (int r = 0; r < 4; ++r) {
     const int j = 64 * g + rg + 16 * r;
     const size_t off = ((size_t)bh * Nbp + j) * kHeadDim + 8 * c16;
-    *reinterpret_cast<uint2*>(kbar8 + off) = j < s.Nb ? codes8(vals[r], sc) : make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(kbar8 + off) = (j < s.Nb && m > 0.f) ? codes8(vals[r], m) : make_uint2(0u, 0u);
     if (j >= s.Nb) *reinterpret_cast<uint2*>(vbar8 + off) = make_uint2(0u, 0u);
   }
 }

@@ -1,25 +1,20 @@
 """GPU parity of the FP8 (E4M3) + ExpCast entry points against the FP8 reference (oracle/fp8_oracle.py).
 
-The kernels follow the reference's arithmetic: the same E4M3 operands, the same ExpCast codes up to
-an exact binade shift of the pivot (both pivots are integers in base 2), the denominators as sums of
-the decoded weights.  ExpCast is discontinuous, though: one code step changes a weight by 2^(1/8)
-(9 %), and a score that lies within the products' rounding error of a code boundary can round to
-either neighbour.  Hence two kinds of check:
+The kernels follow the reference's arithmetic: the same E4M3 operands (the quantiser keeps exact
+midpoints exact), the same ExpCast codes up to an exact binade shift of the pivot (both pivots are
+integers in base 2), the denominators as sums of the decoded weights; an FP32 model of the kernels
+matches the reference to FP32 rounding on the CPU (tests/test_fp8_algorithm_model.py).  A code can
+still differ where a score lies within FP32 rounding of a code boundary (a handful per 10^5
+scores), so every case uses the BF16 path's tolerances (max-abs 2e-2, relative l2 5e-3).  The
+exact-products case (sparse +-1 Q and K: every product and partial sum exact in any accumulator,
+every code line 2.9e-2 or more from a rounding boundary) leaves no room even for that.
 
-* exact products: Q and K sparse +-1 vectors (16 nonzeros of 128), so every E4M3 product and every
-  partial sum is exact in any accumulator and every code line 8u + 55.65 stays 2.9e-2 or more from a
-  rounding boundary (whatever the integer pivot); the kernels must then match the reference within
-  the BF16 tolerances (max-abs 2e-2, relative l2 5e-3);
-* random inputs: code flips allowed.  The bound (relative l2 2e-2, max-abs 4e-2) is twice what the
-  first B200 run measured on n300 (1.1e-2 relative l2, 1.9e-2 max-abs) and covers what perturbing
-  the reference's key operands by 2^-14 .. 2^-10 relative does to it (5e-3 .. 8e-3 relative l2):
-  reduced-precision accumulation of the E4M3 products; the output must also stay at least three
-  times closer to the FP8 reference than to the BF16 one.
-
-These kernels had their first run (n300, both entry points, bounds-checked library: status 0,
-1.1e-2 relative l2 against this reference, 5.4e-2 against the BF16 path); until the whole module
-has run on a GPU it is skipped unless SOL_FP8_GPU=1 is set, so that an unattended GPU suite does
-not make that run.
+First B200 run (n300, one head, both entry points, bounds-checked library): device status 0,
+1.08e-2 relative l2 from this reference and 5.4e-2 from the BF16 path, matching the FP32 model of
+the kernels to four digits; the 1 % came from the quantiser's former order x / (max / 448), which
+rounds exact E4M3 midpoints the wrong way, and is fixed.  Until the module has run once more under
+supervision it is skipped unless SOL_FP8_GPU=1 is set, so that an unattended GPU suite does not
+make that run.
 """
 import os
 import zlib
@@ -39,8 +34,8 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(os.environ.get("SOL_FP8_GPU") != "1",
                                  reason="FP8 kernels not yet run on a GPU: first run is a supervised call")]
 
-FP8_MAX_ABS = 4e-2     # random inputs: ExpCast code flips allowed (module docstring)
-FP8_REL_L2 = 2e-2
+FP8_MAX_ABS = 2e-2     # the BF16 path's tolerances (module docstring)
+FP8_REL_L2 = 5e-3
 
 REF = {"sol_attn": f8.sol_attn_fp8, "sol_attn2": f8.sol_attn2_fp8}
 GPU = {"sol_attn": lambda *a, **kw: sa.sol_attn_fwd_fp8(*a, **kw),
