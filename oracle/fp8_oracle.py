@@ -35,6 +35,8 @@ R19 ExpCast gives every weight of the shared softmax, exact tokens and surrogate
     (u <= 8, the largest weight coded 112..120), the same range an online pivot moved only when the
     running maximum exceeds it by more than 8 keeps.
 R20 An all-zero quantisation block keeps scale 1 and zero codes.
+R22 The quotient X / s_X is the exact real number 448 X / max|X| rounded to E4M3 (nearest, ties to
+    even); it is evaluated in that form (exact products for BF16 inputs), not as X / fl(s_X).
 R21 Sol-Attn2 under FP8: the exact branch as above (E4M3 operands, ExpCast weights against the
     integer pivot ceil(max exact score / ln 2) - 8); the complementary tail's Z_a, mu_a, nu_a are
     those of the BF16 path (computed from the original inputs: the tail is not a product of the
@@ -86,11 +88,26 @@ def expcast(u) -> np.ndarray:
 
 
 def quantize(x) -> tuple[np.ndarray, float]:
-    """One E4M3 scale for the whole array: (s_X X_8 as FP64, s_X)."""
+    """One E4M3 scale for the whole array: (s_X X_8 as FP64, s_X).
+
+    X / s_X is evaluated as 448 X / max|X|, the same real number: for inputs with few mantissa bits
+    (BF16) the product is exact and the quotient exact whenever it is representable, so a value
+    exactly halfway between two E4M3 numbers stays halfway and rounds to even, as the definition
+    asks.  X / fl(max|X| / 448) carries the rounding of s_X and can land one unit off the midpoint
+    (R22)."""
     x = np.asarray(x, dtype=np.float64)
     amax = float(np.abs(x).max()) if x.size else 0.0
-    s = amax / E4M3_MAX if amax > 0 else 1.0
-    return s * e4m3_round(x / s), s
+    return quantize_with_max(x, amax)
+
+
+def quantize_with_max(x, amax: float) -> tuple[np.ndarray, float]:
+    """(s X_8, s) with s = amax / 448 for an array whose scale comes from amax (the max of a larger
+    set, e.g. the head's V for the value means); amax = 0 gives scale 1 and zero codes (R20)."""
+    x = np.asarray(x, dtype=np.float64)
+    if amax <= 0:
+        return np.zeros_like(x), 1.0
+    s = amax / E4M3_MAX
+    return s * e4m3_round(x * E4M3_MAX / amax), s
 
 
 def quantize_blocks(x_bh: np.ndarray, block: int = orc.BLOCK) -> np.ndarray:
@@ -128,12 +145,12 @@ def sol_attn_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, kbar8, vbar8, counts):
     return num / den[:, None]
 
 
-def surrogate_operands_fp8(Kbar, Vhat, counts, v_scale: float):
+def surrogate_operands_fp8(Kbar, Vhat, counts, v_amax: float):
     """E4M3 compressed keys and values of one head (R18): Kbar per 64 consecutive block means,
-    Vbar = Vhat / n with the head's V scale."""
+    Vbar = Vhat / n with the head's V scale (v_amax = max |V| of the head)."""
     kbar8 = quantize_blocks(Kbar)
     vbar = Vhat / counts[:, None]
-    return kbar8, v_scale * e4m3_round(vbar / v_scale)
+    return kbar8, quantize_with_max(vbar, v_amax)[0]
 
 
 def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None):
@@ -150,8 +167,8 @@ def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0
             r = orc._routing_for_head(q_bh, k_bh, tau, sink)
             masks[b, h] = r["mask"]
             q8, k8 = quantize_blocks(q_bh), quantize_blocks(k_bh)
-            v8, sv = quantize(v_bh)
-            kbar8, vbar8 = surrogate_operands_fp8(r["Kbar"], orc.block_sums(v_bh), r["counts"], sv)
+            v8 = quantize(v_bh)[0]
+            kbar8, vbar8 = surrogate_operands_fp8(r["Kbar"], orc.block_sums(v_bh), r["counts"], float(np.abs(v_bh).max()))
             for i in (range(Nb) if qblocks is None else qblocks):
                 lo, hi = orc.block_range(i, N)
                 out[b, lo:hi, h] = sol_attn_fp8_rows(q8[lo:hi], k8, v8, r["mask"][i], kbar8, vbar8, r["counts"])

@@ -36,6 +36,17 @@ def test_expcast_powers_of_two_and_error_bound():
     assert rel.max() < 0.075                                           # piecewise-linear mantissa
 
 
+def test_quantizer_rounds_exact_midpoints_to_even():
+    # max 3.8125 (BF16): 448 x / max = -168 exactly for x = -1.4296875, halfway between -160 and -176;
+    # ties go to even (-160 = -1.25 * 2^7).  x / (max / 448) in FP64 gives -168.00000000000003.
+    x = np.array([-1.4296875, 0.08935546875, 3.8125])
+    xq, s = f8.quantize(x)
+    np.testing.assert_array_equal(xq / s, [-160.0, 10.0, 448.0])
+    assert f8.e4m3_round(-1.4296875 / (3.8125 / 448.0)) == -176.0          # the other order's result
+    ref = torch.tensor(x * 448.0 / 3.8125, dtype=torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(xq / s, ref)
+
+
 def test_quantizer_extremes():
     g = np.random.default_rng(1)
     x = g.standard_normal((64, 128)) * 3.0
@@ -73,12 +84,12 @@ def test_surrogate_operands_are_quantised_like_keys_and_values():
     counts = np.full(150, 64)
     counts[-1] = 17
     Vhat = g.standard_normal((150, 128)) * counts[:, None]
-    kbar8, vbar8 = f8.surrogate_operands_fp8(Kbar, Vhat, counts, v_scale=0.01)
+    kbar8, vbar8 = f8.surrogate_operands_fp8(Kbar, Vhat, counts, v_amax=4.48)
     for a, b in ((0, 64), (64, 128), (128, 150)):
         s = np.abs(Kbar[a:b]).max() / 448.0
         np.testing.assert_array_equal(kbar8[a:b], s * f8.e4m3_round(Kbar[a:b] / s))
     vbar = Vhat / counts[:, None]
-    np.testing.assert_array_equal(vbar8, 0.01 * f8.e4m3_round(vbar / 0.01))
+    np.testing.assert_array_equal(vbar8, (4.48 / 448.0) * f8.e4m3_round(vbar * 448.0 / 4.48))
     assert np.abs(vbar8 - vbar).max() <= 2.0 ** -4 * np.abs(vbar).max()
 
 

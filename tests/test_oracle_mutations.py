@@ -143,14 +143,22 @@ def _fp8_surrogate_sums(q8_rows, k8_bh, v8_bh, mask_row, kbar8, vbar8, counts):
     return _orig_fp8_rows(q8_rows, k8_bh, v8_bh, mask_row, kbar8, vbar8 * counts[:, None], counts)
 
 
-def _surrogate_one_key_scale(Kbar, Vhat, counts, v_scale):
-    _, vbar8 = _orig_surrogate(Kbar, Vhat, counts, v_scale)
+def _surrogate_one_key_scale(Kbar, Vhat, counts, v_amax):
+    _, vbar8 = _orig_surrogate(Kbar, Vhat, counts, v_amax)
     return f8.quantize(Kbar)[0], vbar8
 
 
-def _surrogate_sums_quantised(Kbar, Vhat, counts, v_scale):
-    kbar8, _ = _orig_surrogate(Kbar, Vhat, counts, v_scale)
-    return kbar8, v_scale * f8.e4m3_round(Vhat / v_scale)
+def _surrogate_sums_quantised(Kbar, Vhat, counts, v_amax):
+    kbar8, _ = _orig_surrogate(Kbar, Vhat, counts, v_amax)
+    return kbar8, f8.quantize_with_max(Vhat, v_amax)[0]
+
+
+def _quantize_scale_first(x):
+    # X / fl(max / 448): the order that rounds exact midpoints the wrong way
+    x = np.asarray(x, dtype=np.float64)
+    amax = float(np.abs(x).max())
+    s = amax / 448.0 if amax > 0 else 1.0
+    return s * f8.e4m3_round(x / s), s
 
 
 _orig_surrogate = f8.surrogate_operands_fp8
@@ -184,6 +192,7 @@ FP8_CASES = [
      fp8pins.test_expcast_powers_of_two_and_error_bound),
     ("expcast", _expcast_no_clip, fp8pins.test_expcast_powers_of_two_and_error_bound),
     ("quantize", _quantize_no_scale, fp8pins.test_quantizer_extremes),
+    ("quantize", _quantize_scale_first, fp8pins.test_quantizer_rounds_exact_midpoints_to_even),
     ("sol_attn_fp8_rows", _fp8_surrogate_sums, fp8pins.test_fp8_forward_with_zero_queries_averages_the_values),
     ("surrogate_operands_fp8", _surrogate_one_key_scale,
      fp8pins.test_surrogate_operands_are_quantised_like_keys_and_values),
