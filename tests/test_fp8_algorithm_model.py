@@ -81,10 +81,10 @@ class _Half:
         self.l = F(self.l + p.sum(dtype=F))
 
 
-def _model_head(q, k, v, tau, sol2):
+def _model_head(q, k, v, tau, sol2, sink_start=-1, sink_tokens=0):
     N = q.shape[0]
     Nb = orc.num_blocks(N)
-    r = orc._routing_for_head(q, k, tau, orc.sink_block_flags(N, -1, 0))
+    r = orc._routing_for_head(q, k, tau, orc.sink_block_flags(N, sink_start, sink_tokens))
     mask = r["mask"]
     q32, k32, v32 = (x.astype(F) for x in (q, k, v))
     q8, sq = _quant_rows(q32, 64)
@@ -148,12 +148,13 @@ def _model_head(q, k, v, tau, sol2):
 
 
 @pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
-@pytest.mark.parametrize("N,tau,seed", [(300, 1.0, 3), (700, 0.5, 4)])
-def test_fp32_model_of_the_kernel_matches_the_reference(lib, entry, N, tau, seed):
+@pytest.mark.parametrize("N,tau,seed,ss,st", [(300, 1.0, 3, -1, 0), (700, 0.5, 4, -1, 0), (1000, 1.5, 6, 300, 200)],
+                         ids=["n300", "n700", "n1000_interior_sink"])
+def test_fp32_model_of_the_kernel_matches_the_reference(lib, entry, N, tau, seed, ss, st):
     q, k, v = iid_qkv(1, N, 1, seed=seed)
     qh, kh, vh = (orc.head_slice(t, 0, 0) for t in (q, k, v))
-    model = _model_head(qh, kh, vh, tau, entry == "sol_attn2")
-    ref = (f8.sol_attn_fp8 if entry == "sol_attn" else f8.sol_attn2_fp8)(q, k, v, tau)["out"][0, :, 0]
+    model = _model_head(qh, kh, vh, tau, entry == "sol_attn2", ss, st)
+    ref = (f8.sol_attn_fp8 if entry == "sol_attn" else f8.sol_attn2_fp8)(q, k, v, tau, ss, st)["out"][0, :, 0]
     # FP32 rounding of the scores can flip a code where a score lies within ~1e-6 of a rounding
     # boundary (3 of 255,248 scores of the N = 700 case lie within 1e-5): a flip moves one weight by
     # 2^(1/8) and the result by a few 1e-5; a systematic difference (a pivot or scale error, the old
