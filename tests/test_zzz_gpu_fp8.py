@@ -157,3 +157,21 @@ def test_fp8_precision_option_and_varlen_match_the_fp8_entry_points():
         if s1 > s0:
             one = sa.sol_attn_fwd_fp8(q[:, s0:s1].contiguous(), k[:, s0:s1].contiguous(), v[:, s0:s1].contiguous(), 1.0)
             assert torch.equal(pv[s0:s1], one[0])
+
+
+@pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
+@pytest.mark.parametrize("N,tau,seed,ss,st", [(300, 1.0, 3, -1, 0), (1000, 1.5, 6, 300, 200)], ids=["n300", "n1000_sink"])
+def test_fp8_kernel_matches_its_fp32_model(entry, N, tau, seed, ss, st):
+    # the FP32 model (tests/test_fp8_algorithm_model.py) follows the kernels' arithmetic step by
+    # step; only the order of the FP32 sums differs, so both round the same values to BF16 except
+    # where a score sits within FP32 rounding of a code boundary (a handful of codes per 10^5
+    # scores flip, each moving one key's weight by 2^(1/8)).  Relative l2 1e-3 is below the BF16
+    # rounding floor against the FP64 reference (1.65e-3); a systematic slip gives 1e-2.
+    from tests.test_fp8_algorithm_model import _model_head
+
+    q, k, v = iid_qkv(1, N, 1, seed=seed)
+    gout, _ = _run(entry, q, k, v, tau, ss, st)
+    model = _model_head(*(orc.head_slice(t, 0, 0) for t in (q, k, v)), tau, entry == "sol_attn2", ss, st)
+    model = torch.tensor(model).to(torch.bfloat16).float().numpy()
+    d = gout[0, :, 0] - model
+    assert np.abs(d).max() <= 2e-2 and np.linalg.norm(d) / np.linalg.norm(model) <= 1e-3
