@@ -32,8 +32,12 @@ R19 ExpCast gives every weight of the shared softmax, exact tokens and surrogate
     2^-6 of the pivot (subnormal codes and the clip at 0).  The code range [0, 120] spans
     u in [-6.96, 8.04]: a pivot at the maximum would leave half of it unused and drop every weight
     below 2^-7 of the maximum, so the reference takes the pivot ceil(row max) - 8 in base 2
-    (u <= 8, the largest weight coded 112..120), the same range an online pivot moved only when the
-    running maximum exceeds it by more than 8 keeps.
+    (u <= 8, the largest weight coded 112..120), the range an online pivot moved only when the
+    running maximum exceeds it by more than 8 keeps.  An online pass differs in one respect: a weight
+    coded before the pivot moved keeps its code, while this final pivot clips every weight more than
+    ~7 binades below it (about 15 binades below the row maximum).  The two agree whenever no such
+    weight exists, which covers ordinary inputs; a row whose maximum jumps by 14 binades after many
+    small scores (keys scaled by 0.25, then by 3) differs by ~6e-3 relative l2.
 R20 An all-zero quantisation block keeps scale 1 and zero codes.
 R22 The quotient X / s_X is the exact real number 448 X / max|X| rounded to E4M3 (nearest, ties to
     even); it is evaluated in that form (exact products for BF16 inputs), not as X / fl(s_X).
