@@ -170,8 +170,21 @@ def test_fp8_kernel_matches_its_fp32_model(entry, N, tau, seed, ss, st):
     from tests.test_fp8_algorithm_model import _model_head
 
     q, k, v = iid_qkv(1, N, 1, seed=seed)
-    gout, _ = _run(entry, q, k, v, tau, ss, st)
+    gout, (qd, kd, _) = _run(entry, q, k, v, tau, ss, st)
     model = _model_head(*(orc.head_slice(t, 0, 0) for t in (q, k, v)), tau, entry == "sol_attn2", ss, st)
     model = torch.tensor(model).to(torch.bfloat16).float().numpy()
-    d = gout[0, :, 0] - model
-    assert np.abs(d).max() <= 2e-2 and np.linalg.norm(d) / np.linalg.norm(model) <= 1e-3
+    rows = model_rows_with_agreeing_masks(qd, kd, q, k, tau, ss, st)
+    d = gout[0, rows, 0] - model[rows]
+    assert np.abs(d).max() <= 2e-2 and np.linalg.norm(d) / np.linalg.norm(model[rows]) <= 1e-3
+
+
+def model_rows_with_agreeing_masks(qd, kd, q, k, tau, ss=-1, st=0):
+    """Token rows whose query block has the same exact set on the GPU router as in the reference's
+    routing, which the FP32 model uses (a pair within the 1e-3 proxy margin may differ)."""
+    N = q.shape[1]
+    gmask, _ = sa.debug_route(qd, kd, tau, ss, st)
+    full = orc.routing(q, k, tau, ss, st)
+    skip = check_mask(gmask.cpu().numpy(), full, orc.sink_block_flags(N, ss, st))
+    rows = ~np.repeat(skip[0, 0], 64)[:N]
+    assert rows.mean() >= 0.9
+    return rows
