@@ -1,16 +1,18 @@
 """GPU: rows whose running maximum jumps mid-row, so that the fused kernels' lazy rescaling runs.
 
-Keys of the first half of the sequence are scaled by 0.25 and of the second half by 3, so a row's
-maximum grows by about 14 binades after its early tiles: the BF16 kernel's reference maximum and
-the FP8 kernel's integer pivot both move (more than 8 binades), and O (and the FP8 row sums) are
-rescaled.  Random inputs almost never do this.
+Keys of the first half of the sequence are scaled by 0.25 and of the second half by 2, so a row's
+maximum grows by about 9 binades after its early tiles: the BF16 kernel's reference maximum moves
+(it moves only past 8 binades: in 567 of the 2048 row halves here) and the FP8 kernel's integer
+pivot moves (about 4300 times), and O (and the FP8 row sums) are rescaled.  Random inputs almost
+never do this.  (A scale of 3 moves nearly every row but makes attention so peaked that outputs
+reach 3.4, where BF16 rounding alone uses 40 % of the max-abs tolerance.)
 
 * BF16: rescaling by exact powers of two changes nothing but FP32 rounding, so the kernel must match
   the FP64 reference within the usual tolerances.
 * FP8: the pivot is online, as in the pages' description of ExpCast, so weights coded before the
   pivot moved keep codes the final pivot would clip (they sit ~14 binades below the row maximum);
-  the reference codes every weight against the final pivot (reading R19) and drops them, which here
-  moves the result by ~6e-3 relative l2.  The kernels are therefore compared with their FP32 model,
+  the reference codes every weight against the final pivot (reading R19) and drops them, which on
+  such rows moves the result by several 1e-3 relative l2.  The kernels are therefore compared with their FP32 model,
   which follows the same online pivots (tests/test_fp8_algorithm_model.py).
 """
 import numpy as np
@@ -31,7 +33,7 @@ def _inputs():
     q, k, v = iid_qkv(1, N, 1, seed=31)
     k = k.float()
     k[:, : N // 2] *= 0.25
-    k[:, N // 2:] *= 3.0
+    k[:, N // 2:] *= 2.0
     return q, k.to(torch.bfloat16), v
 
 
