@@ -219,7 +219,7 @@ def sol_attn2_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 
             q_bh, k_bh, v_bh = orc.head_slice(q, b, h), orc.head_slice(k, b, h), orc.head_slice(v, b, h)
             r = orc._routing_for_head(q_bh, k_bh, tau, sink)
             masks[b, h] = r["mask"]
-            counts, kg, vg = orc.key_groups(k_bh, v_bh, q_bh.mean(axis=0))
+            counts, kg, vg = orc.key_groups(k_bh, v_bh, orc.group_direction(q_bh, k_bh))
             qbar_anchor = orc.block_means(q_bh, orc.ANCHOR)
             q8, k8 = quantize_blocks(q_bh), quantize_blocks(k_bh)
             v8 = quantize(v_bh)[0]

@@ -291,6 +291,14 @@ def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qb
 # Sol-Attn2 complementary tail: [Sol2] "Routing and complementary approximation", readings R9-R12.
 # ----------------------------------------------------------------------------------------------
 
+def group_direction(q_bh: np.ndarray, k_bh: np.ndarray) -> np.ndarray:
+    """The direction the keys are split on ([Sol2] "Routing and complementary approximation": the
+    mean-query direction), per reading R10: the mean of all queries of the (batch, head), one
+    direction shared by every anchor and query block.  ``k_bh`` is unused (it is part of the
+    signature so that readings based on the keys can be compared in the tests)."""
+    return q_bh.mean(axis=0)
+
+
 def key_groups(k_bh: np.ndarray, v_bh: np.ndarray, u: np.ndarray):
     """Two content groups per key block, split by the key projection on direction u (R10).
 
@@ -357,25 +365,28 @@ def sol_attn2_rows(q_rows, row0, k_bh, v_bh, mask_row, counts, kg, vg, qbar_anch
 
 def sol_attn2(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None,
               extra_sinks=()):
-    """Sol-Attn2 forward (complementary tail). Same return convention as :func:`sol_attn`."""
+    """Sol-Attn2 forward (complementary tail). Same return convention as :func:`sol_attn`, plus
+    ``group_counts`` [B, H, Nb, 2]: n_g of the two key groups of every block (group 1 = the keys
+    whose projection on the direction lies strictly above the block mean's)."""
     B, N, H, _ = q.shape
     Nb = num_blocks(N)
     sink = sink_block_flags(N, sink_start, sink_tokens, extra_sinks)
     out = np.full((B, N, H, HEAD_DIM), np.nan)
     masks = np.zeros((B, H, Nb, Nb), dtype=bool)
+    group_counts = np.zeros((B, H, Nb, 2), dtype=np.int64)
     pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
     for b, h in pairs:
         q_bh, k_bh, v_bh = head_slice(q, b, h), head_slice(k, b, h), head_slice(v, b, h)
         r = _routing_for_head(q_bh, k_bh, tau, sink)
         masks[b, h] = r["mask"]
-        u = q_bh.mean(axis=0)
-        counts, kg, vg = key_groups(k_bh, v_bh, u)
+        counts, kg, vg = key_groups(k_bh, v_bh, group_direction(q_bh, k_bh))
+        group_counts[b, h] = counts
         qbar_anchor = block_means(q_bh, ANCHOR)
         for i in _row_subset(N, qblocks):
             lo, hi = block_range(i, N)
             out[b, lo:hi, h] = sol_attn2_rows(q_bh[lo:hi], lo, k_bh, v_bh, r["mask"][i], counts, kg, vg,
                                               qbar_anchor)
-    return dict(out=out, mask=masks)
+    return dict(out=out, mask=masks, group_counts=group_counts)
 
 
 def dense_rows(q, k, v, q_start: int, q_tokens: int):

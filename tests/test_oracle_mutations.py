@@ -86,6 +86,76 @@ def _diag_without_mean(Qbar, Kbar, tau):
     return 0.0 * mu, sigma, tau * sigma
 
 
+def _direction_key_mean(q_bh, k_bh):
+    return k_bh.mean(axis=0)
+
+
+def _direction_first_anchor(q_bh, k_bh):
+    return q_bh[: orc.ANCHOR].mean(axis=0)
+
+
+def _direction_flipped(q_bh, k_bh):
+    return -q_bh.mean(axis=0)
+
+
+_orig_key_groups = orc.key_groups
+
+
+def _ties_upper(k_bh, v_bh, u):
+    N = k_bh.shape[0]
+    Nb = orc.num_blocks(N)
+    counts, kg, vg = np.zeros((Nb, 2), np.int64), np.zeros((Nb, 2, orc.HEAD_DIM)), np.zeros((Nb, 2, orc.HEAD_DIM))
+    for j in range(Nb):
+        a, b = orc.block_range(j, N)
+        proj = (k_bh[a:b] @ u).astype(np.float32)
+        upper = proj >= np.float32(k_bh[a:b].mean(axis=0) @ u)
+        for g, sel in ((0, ~upper), (1, upper)):
+            counts[j, g] = int(sel.sum())
+            if counts[j, g]:
+                kg[j, g], vg[j, g] = k_bh[a:b][sel].mean(axis=0), v_bh[a:b][sel].mean(axis=0)
+    return counts, kg, vg
+
+
+def _groups_median_split(k_bh, v_bh, u):
+    # equal halves (split at the median projection) instead of the block mean's projection
+    N = k_bh.shape[0]
+    Nb = orc.num_blocks(N)
+    counts, kg, vg = np.zeros((Nb, 2), np.int64), np.zeros((Nb, 2, orc.HEAD_DIM)), np.zeros((Nb, 2, orc.HEAD_DIM))
+    for j in range(Nb):
+        a, b = orc.block_range(j, N)
+        order = np.argsort(k_bh[a:b] @ u, kind="stable")
+        half = (b - a) // 2
+        for g, sel in ((0, order[:half]), (1, order[half:])):
+            counts[j, g] = len(sel)
+            if len(sel):
+                kg[j, g], vg[j, g] = k_bh[a:b][sel].mean(axis=0), v_bh[a:b][sel].mean(axis=0)
+    return counts, kg, vg
+
+
+def _sol_attn2_per_query_block_direction(q, k, v, tau, sink_start=-1, sink_tokens=0, qblocks=None, heads=None,
+                                         extra_sinks=()):
+    # the reading the oracle rejects: every query block splits the keys on its own mean query
+    B, N, H, _ = q.shape
+    Nb = orc.num_blocks(N)
+    sink = orc.sink_block_flags(N, sink_start, sink_tokens, extra_sinks)
+    out = np.full((B, N, H, orc.HEAD_DIM), np.nan)
+    masks = np.zeros((B, H, Nb, Nb), dtype=bool)
+    group_counts = np.zeros((B, H, Nb, 2), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            q_bh, k_bh, v_bh = orc.head_slice(q, b, h), orc.head_slice(k, b, h), orc.head_slice(v, b, h)
+            r = orc._routing_for_head(q_bh, k_bh, tau, sink)
+            masks[b, h] = r["mask"]
+            qbar_anchor = orc.block_means(q_bh, orc.ANCHOR)
+            for i in range(Nb):
+                lo, hi = orc.block_range(i, N)
+                counts, kg, vg = orc.key_groups(k_bh, v_bh, q_bh[lo:hi].mean(axis=0))
+                out[b, lo:hi, h] = orc.sol_attn2_rows(q_bh[lo:hi], lo, k_bh, v_bh, r["mask"][i], counts, kg, vg,
+                                                      qbar_anchor)
+            group_counts[b, h] = orc.key_groups(k_bh, v_bh, orc.group_direction(q_bh, k_bh))[0]
+    return dict(out=out, mask=masks, group_counts=group_counts)
+
+
 CASES = [
     ("block_sums", _value_means_not_sums,
      lambda: pins.test_identical_unselected_keys_make_the_approximation_exact(448, "sol_attn")),
@@ -106,6 +176,12 @@ CASES = [
     ("dense_rows", _dense_rows_one_short, pins.test_dense_rows_match_library_attention),
     ("dense_rows", _dense_rows_unscaled, pins.test_dense_rows_match_library_attention),
     ("threshold_diag", _diag_without_mean, pins.test_diagonal_estimator_equals_exact_when_key_covariance_is_diagonal),
+    ("group_direction", _direction_key_mean, pins.test_hand_expanded_sol_attn2_split_direction),
+    ("group_direction", _direction_first_anchor, pins.test_hand_expanded_sol_attn2_split_direction),
+    ("group_direction", _direction_flipped, pins.test_hand_expanded_sol_attn2_split_direction),
+    ("key_groups", _ties_upper, pins.test_hand_expanded_sol_attn2_split_direction),
+    ("key_groups", _groups_median_split, pins.test_hand_expanded_sol_attn2_split_direction),
+    ("sol_attn2", _sol_attn2_per_query_block_direction, pins.test_hand_expanded_sol_attn2_split_direction),
 ]
 
 

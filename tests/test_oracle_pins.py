@@ -231,6 +231,70 @@ def test_hand_expanded_sol_attn2():
         np.testing.assert_allclose(r["out"][0, row, 0], expect, rtol=1e-11, atol=1e-14)
 
 
+# ---------------------------------------------------------------- Sol-Attn2 split direction
+
+def _direction_case():
+    """N = 192 (3 blocks), H = 1, in the e1-e2-e3 space.  Anchor bases (tokens 32a .. 32a + 31):
+    (1, 2, 0), (1, 0, 0) | (1, -1, 0), (1, -1, 0) | (1, 0, 3), (1, 0, 3), plus +-0.25 e1 alternating
+    inside each anchor (zero mean, so every anchor mean is its base).  The mean query is then
+    u = (1, 0, 1), while query block 0's mean is (1, 1, 0), query block 2's is (1, 0, 3), anchor 0's
+    is (1, 2, 0) and the keys' mean points elsewhere again: each candidate direction splits the tail
+    blocks differently.  Tail blocks (tau huge: only |i - j| <= 1 is exact):
+      key block 2 (tail of query block 0): 16 x P = (1, 0, 1) (projection on u: 2), 8 x M = (-2, 0, -2)
+        (-4), 20 x (1, 0, -1) and 20 x (0, 1, 0) (both 0, exactly the block mean's projection);
+      key block 0 (tail of query block 2): 12 x A = (2, 1, 0) (2), 8 x (0, 0, -3) (-3), 44 x (0, 2, 0) (0).
+    Types are interleaved by a seeded permutation; values are random."""
+    g = np.random.default_rng(29)
+    N = 192
+    q = np.zeros((1, N, 1, D))
+    bases = [(1, 2, 0), (1, 0, 0), (1, -1, 0), (1, -1, 0), (1, 0, 3), (1, 0, 3)]
+    for a, base in enumerate(bases):
+        q[0, 32 * a: 32 * a + 32, 0, :3] = base
+    eps = np.where(np.arange(N) % 2 == 0, 0.25, -0.25)
+    q[0, :, 0, 0] += eps
+    k = np.zeros((1, N, 1, D))
+    blk2 = [(1, 0, 1)] * 16 + [(-2, 0, -2)] * 8 + [(1, 0, -1)] * 20 + [(0, 1, 0)] * 20
+    blk0 = [(2, 1, 0)] * 12 + [(0, 0, -3)] * 8 + [(0, 2, 0)] * 44
+    p2, p0 = g.permutation(64), g.permutation(64)
+    k[0, 128:, 0, :3] = np.array(blk2, float)[p2]
+    k[0, :64, 0, :3] = np.array(blk0, float)[p0]
+    k[0, 64:128, 0, :3] = 0.5 * g.standard_normal((64, 3))
+    upper2 = p2 < 16          # the P keys: the only keys of block 2 strictly above the split
+    upper0 = p0 < 12          # the A keys of block 0
+    v = g.standard_normal((1, N, 1, D))
+    return dict(q=q, k=k, v=v, eps=eps, bases=np.array(bases, float), upper={2: upper2, 0: upper0})
+
+
+def test_hand_expanded_sol_attn2_split_direction():
+    """[Sol2] "Routing and complementary approximation": each unselected block splits into two groups
+    by key projection on the mean-query direction (reading R10: the mean of all queries of the
+    head; keys strictly above the block mean's projection form group 1).  The groups of both tail
+    blocks are written out by hand from the construction, and the outputs of rows of both tail
+    query blocks are expanded from them.  The key mean, a query block's or an anchor's mean, or
+    -u would each group the keys differently (and the tied keys pin the side ties fall on)."""
+    h = _direction_case()
+    r = orc.sol_attn2(h["q"], h["k"], h["v"], tau=1e6)
+    assert r["mask"][0, 0].tolist() == [[True, True, False], [True, True, True], [False, True, True]]
+    assert r["group_counts"][0, 0, 2].tolist() == [48, 16]
+    assert r["group_counts"][0, 0, 0].tolist() == [52, 12]
+    q, k, v = h["q"][0, :, 0], h["k"][0, :, 0], h["v"][0, :, 0]
+    for qi, tail, exact in ((0, 2, slice(0, 128)), (2, 0, slice(64, 192))):
+        kb, vb = k[64 * tail: 64 * tail + 64], v[64 * tail: 64 * tail + 64]
+        up = h["upper"][tail]
+        groups = [(int((~up).sum()), kb[~up].mean(0), vb[~up].mean(0)), (int(up.sum()), kb[up].mean(0), vb[up].mean(0))]
+        for row in (64 * qi, 64 * qi + 1, 64 * qi + 33, 64 * qi + 62):
+            qa = np.zeros(D)
+            qa[:3] = h["bases"][row // 32]
+            w = [n * math.exp(S * float(qa @ kg)) for n, kg, _ in groups]
+            Z = sum(w)
+            mu = sum(wi * kg for wi, (_, kg, _) in zip(w, groups)) / Z
+            nu = sum(wi * vg for wi, (_, _, vg) in zip(w, groups)) / Z
+            Zhat = Z * math.exp(S * float((q[row] - qa) @ mu))
+            we = np.exp(S * (k[exact] @ q[row]))
+            expect = (we @ v[exact] + Zhat * nu) / (we.sum() + Zhat)
+            np.testing.assert_allclose(r["out"][0, row, 0], expect, rtol=1e-11, atol=1e-14)
+
+
 # ---------------------------------------------------------------------------- Sol-Attn2 groups
 
 def test_group_counts_preserve_block_mass():
