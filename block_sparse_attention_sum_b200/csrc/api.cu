@@ -290,13 +290,15 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
       cudaMemsetAsync(d.stats + 1, 0xff, sizeof(unsigned long long), st) != cudaSuccess ||
       cudaMemsetAsync(d.stats + 2, 0, sizeof(unsigned long long), st) != cudaSuccess)
     return fail(SOL_ERR_LAUNCH, "stats reset failed");
+  // every caller reaches the tensor-map encoder through here, so look it up here
+  int rc = get_encode();
+  if (rc) return rc;
   Work ww = w;
   ww.stats = d.stats;
   launch_summary(q, k, v, s, ww, anchors, st);
   launch_kstats(s, ww, st);
   launch_thresh(s, ww, tau, diag, st);
   CUtensorMap rmaps[4];
-  int rc;
   if ((rc = encode_rows(&rmaps[0], w.qbar_hi, s.Nb, s)) || (rc = encode_rows(&rmaps[1], w.qbar_lo, s.Nb, s)) ||
       (rc = encode_rows(&rmaps[2], w.kbar_h, s.Nb, s)) || (rc = encode_rows(&rmaps[3], w.kbar_lo, s.Nb, s)))
     return rc;

@@ -59,3 +59,28 @@ def test_workspace_limit_reports_alloc_failure():
     out = sa.sol_attn_fwd(q, k, v, 1.0)
     torch.cuda.synchronize()
     assert sa.get_device_status() == 0 and torch.isfinite(out.float()).all()
+
+
+def test_debug_route_as_the_first_call_in_a_fresh_process():
+    # the routing introspection call must set up everything it uses (the tensor-map encoder among
+    # them) when it is the first call of the C ABI a process makes, as __graft_entry__.smoke() does
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import torch\n"
+        "from block_sparse_attention_sum_b200 import sol_attn as sa\n"
+        "from block_sparse_attention_sum_b200.inputs import iid_qkv\n"
+        "q, k, v = (t.cuda() for t in iid_qkv(1, 1024, 2, seed=0))\n"
+        "mask, thr = sa.debug_route(q, k, 1.0)\n"
+        "out = sa.sol_attn_fwd(q, k, v, 1.0)\n"
+        "torch.cuda.synchronize()\n"
+        "assert sa.get_device_status() == 0\n"
+        "assert bool(mask.any()) and bool(torch.isfinite(out.float()).all())\n"
+        "print('ok')\n"
+    )
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, (r.returncode, r.stdout[-2000:], r.stderr[-2000:])
+    assert r.stdout.strip().endswith("ok")
