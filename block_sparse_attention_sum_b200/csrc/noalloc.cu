@@ -21,6 +21,7 @@
 
 #include "attn_fwd.cuh"
 #include "common.cuh"
+#include "ptx.cuh"
 #include "sol_attn.h"
 
 namespace sol {
@@ -77,6 +78,38 @@ size_t na_carve(const Shape& s, unsigned char* base, Work* w) {
   return off;
 }
 
+// Looks up, once per device and with that device current, the device addresses of the file-scope
+// buffers.  cudaGetSymbolAddress also loads this file's module on the device if it is not loaded
+// yet (lazy module loading), and that load is when the driver reserves the 64 MiB region.
+// Caller holds g_na_mu.
+int na_setup(NoAllocDevice** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return na_fail(SOL_ERR_DEVICE, "no current CUDA device");
+  NoAllocDevice& d = g_na[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess || major != 10 ||
+        minor != 0)
+      return na_fail(SOL_ERR_DEVICE, "the current device is not an sm_100 (B200-class) GPU");
+    void* a = nullptr;
+    void* b = nullptr;
+    void* c = nullptr;
+    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess ||
+        cudaGetSymbolAddress(&b, g_noalloc_status) != cudaSuccess ||
+        cudaGetSymbolAddress(&c, g_noalloc_stats) != cudaSuccess || !a || !b || !c) {
+      cudaGetLastError();
+      return na_fail(SOL_ERR_DEVICE, "cudaGetSymbolAddress failed for the scratch region");
+    }
+    d.scratch = static_cast<unsigned char*>(a);
+    d.status = static_cast<int*>(b);
+    d.stats = static_cast<unsigned long long*>(c);
+    d.ready = true;
+  }
+  *out = &d;
+  return SOL_OK;
+}
+
 int na_encode(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, int rank,
               const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
   const cuuint32_t estr[4] = {1, 1, 1, 1};
@@ -121,31 +154,10 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   }
 
   std::lock_guard<std::mutex> lock(g_na_mu);
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return na_fail(SOL_ERR_DEVICE, "no current CUDA device");
-  NoAllocDevice& d = g_na[dev];
-  if (!d.ready) {
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess || major != 10 ||
-        minor != 0)
-      return na_fail(SOL_ERR_DEVICE, "the current device is not an sm_100 (B200-class) GPU");
-    // device addresses of the file-scope buffers on this device (the first call on a device does
-    // this set-up; make that first call before any stream capture)
-    void* a = nullptr;
-    void* b = nullptr;
-    void* c = nullptr;
-    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess ||
-        cudaGetSymbolAddress(&b, g_noalloc_status) != cudaSuccess ||
-        cudaGetSymbolAddress(&c, g_noalloc_stats) != cudaSuccess || !a || !b || !c) {
-      cudaGetLastError();
-      return na_fail(SOL_ERR_DEVICE, "cudaGetSymbolAddress failed for the scratch region");
-    }
-    d.scratch = static_cast<unsigned char*>(a);
-    d.status = static_cast<int*>(b);
-    d.stats = static_cast<unsigned long long*>(c);
-    d.ready = true;
-  }
+  NoAllocDevice* dp = nullptr;
+  int rc0 = na_setup(&dp);
+  if (rc0) return rc0;
+  NoAllocDevice& d = *dp;
 
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult qr;
@@ -222,5 +234,26 @@ extern "C" int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   if (e != cudaSuccess) return na_fail(SOL_ERR_LAUNCH, cudaGetErrorString(e));
   e = cudaGetLastError();
   if (e != cudaSuccess) return na_fail(SOL_ERR_LAUNCH, cudaGetErrorString(e));
+  return SOL_OK;
+}
+
+// Reads and clears the status word the allocation-free call's kernels write (a bounded wait that
+// ran out, a misaligned shared-memory window).  Synchronises `stream` first; copies four bytes to a
+// host variable and clears them with cudaMemset: nothing is allocated.
+extern "C" int sol_attn_noalloc_get_device_status(void* stream) {
+  set_last_error("");
+  std::lock_guard<std::mutex> lock(g_na_mu);
+  NoAllocDevice* d = nullptr;
+  int rc = na_setup(&d);
+  if (rc) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return na_fail(SOL_ERR_LAUNCH, "stream synchronisation failed");
+  int h = 0;
+  if (cudaMemcpy(&h, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(d->status, 0, sizeof(int)) != cudaSuccess)
+    return na_fail(SOL_ERR_LAUNCH, "status read failed");
+  if (h == kDevTimeout) return na_fail(SOL_ERR_TIMEOUT, "a bounded wait inside a kernel ran out");
+  if (h == kDevMisaligned) return na_fail(SOL_ERR_LAUNCH, "shared memory window misaligned; the kernel did not run");
+  if (h == kDevBounds) return na_fail(SOL_ERR_LAUNCH, "a bounds check of the debug build failed (access skipped)");
   return SOL_OK;
 }

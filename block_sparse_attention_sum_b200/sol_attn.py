@@ -33,6 +33,7 @@ EXPORTS = [
     "sol_attn_last_launch_count",
     "sol_attn_release_workspace",
     "sol_attn_fwd_noalloc",
+    "sol_attn_noalloc_get_device_status",
     "sol_attn_fwd_varlen",
     "sol_attn_dense_rows",
     "sol_attn_set_workspace_limit",
@@ -137,6 +138,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_release_workspace.restype = None
     lib.sol_attn_fwd_noalloc.argtypes = fwd_args
     lib.sol_attn_fwd_noalloc.restype = i
+    lib.sol_attn_noalloc_get_device_status.argtypes = [vp]
+    lib.sol_attn_noalloc_get_device_status.restype = i
     lib.sol_attn_dense_rows.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.sol_attn_dense_rows.restype = i
     lib.sol_attn_fwd_varlen.argtypes = [vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int), i, i, f, i, i, op, vp]
@@ -341,6 +344,10 @@ def selftest_wait_timeout(stream=None) -> int:
 
 def get_device_status(stream=None) -> int:
     return load_library().sol_attn_get_device_status(_stream_handle(stream))
+
+
+def noalloc_get_device_status(stream=None) -> int:
+    return load_library().sol_attn_noalloc_get_device_status(_stream_handle(stream))
 
 
 def set_kernel_timing(enable: bool):

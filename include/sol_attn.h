@@ -206,15 +206,28 @@ void sol_attn_release_workspace(void);
  *     scratch exceeds 64 MiB (for example B*H = 32 at N > ~38K tokens) returns SOL_ERR_SHAPE with a
  *     message; use sol_attn_fwd for those.
  *   - The first call on a device (with that device current) looks up the scratch region's device
- *     address; make that first call before any stream capture on the device.
+ *     address.  Under CUDA's default lazy module loading that lookup is also when the driver
+ *     loads this part of the library on the device and reserves the 64 MiB, so make that first
+ *     call (or sol_attn_noalloc_get_device_status) early: before reserving the rest of the
+ *     device's memory and before any stream capture on the device.
  *   - All calls share the one region: calls that overlap on the GPU (different streams, or several
  *     host threads) race and must be serialised by the caller.  The region keeps the last call's
  *     contents; everything a call needs zeroed it clears itself.
- *   - Not covered by sol_attn_last_stats / sol_attn_get_device_status / kernel timing (those
- *     report the pooled-workspace entry points).
+ *   - Device-side failures (a bounded wait that ran out) are reported by
+ *     sol_attn_noalloc_get_device_status, not by sol_attn_get_device_status; sol_attn_last_stats
+ *     and kernel timing report the pooled-workspace entry points only.
  */
 int sol_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
                          int sink_start, int sink_tokens, void* stream);
+
+/*
+ * Status of the allocation-free calls on the current device (the pages have no counterpart).
+ * Synchronises `stream`, then reads and clears the status word that sol_attn_fwd_noalloc's kernels
+ * write: SOL_OK, SOL_ERR_TIMEOUT (a bounded wait inside a kernel ran out: that call's `out` is not
+ * valid) or SOL_ERR_LAUNCH (a kernel found its shared memory misaligned and did not run).  Reads
+ * four bytes into a host variable and clears them with cudaMemset: it allocates nothing.
+ */
+int sol_attn_noalloc_get_device_status(void* stream);
 
 /*
  * Variable-length batch (packed sequences, as the pages' integrations pass them): sequence s holds

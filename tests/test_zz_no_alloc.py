@@ -3,7 +3,8 @@
 Callers that cannot allocate device memory during a call (a caller-managed memory pool, a runtime
 that reserved the device's memory up front) use sol_attn_fwd_noalloc, whose scratch is a fixed
 region inside the library.  This file sorts last so that a run stopping at the first failure has
-already run every other test.
+already run every other test; it passes in a fresh process as well (the first call on the device
+does the region's set-up).
 """
 import ctypes
 
@@ -43,8 +44,11 @@ def test_noalloc_matches_pooled_entry_on_two_calls(case):
         rc = lib.sol_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), q.shape[0],
                                       q.shape[1], q.shape[2], float(tau), ss, st, stream)
         assert rc == 0, lib.sol_attn_last_error()
-        torch.cuda.synchronize()
+        assert lib.sol_attn_noalloc_get_device_status(stream) == 0, lib.sol_attn_last_error()
         _close(out, ref)
+        # the same kernels on the same inputs: the result is the pooled entry point's, bit for bit
+        # (stale scratch from an earlier call would show here first)
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
