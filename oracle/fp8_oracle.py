@@ -157,9 +157,9 @@ def surrogate_operands_fp8(Kbar, Vhat, counts, v_amax: float):
     return kbar8, quantize_with_max(vbar, v_amax)[0]
 
 
-def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None):
+def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, mask_override=None):
     """FP8 + ExpCast Sol-Attn forward.  Returns dict with ``out`` (FP64, NaN for rows not computed)
-    and ``mask`` (the routing of the BF16 path, R18)."""
+    and ``mask`` (the routing of the BF16 path, R18).  ``mask_override`` as in the BF16 oracle."""
     B, N, H, _ = q.shape
     Nb = orc.num_blocks(N)
     sink = orc.sink_block_flags(N, sink_start, sink_tokens)
@@ -173,9 +173,10 @@ def sol_attn_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0
             q8, k8 = quantize_blocks(q_bh), quantize_blocks(k_bh)
             v8 = quantize(v_bh)[0]
             kbar8, vbar8 = surrogate_operands_fp8(r["Kbar"], orc.block_sums(v_bh), r["counts"], float(np.abs(v_bh).max()))
+            use = r["mask"] if mask_override is None else np.asarray(mask_override[b, h], dtype=bool)
             for i in (range(Nb) if qblocks is None else qblocks):
                 lo, hi = orc.block_range(i, N)
-                out[b, lo:hi, h] = sol_attn_fp8_rows(q8[lo:hi], k8, v8, r["mask"][i], kbar8, vbar8, r["counts"])
+                out[b, lo:hi, h] = sol_attn_fp8_rows(q8[lo:hi], k8, v8, use[i], kbar8, vbar8, r["counts"])
     return dict(out=out, mask=masks)
 
 
@@ -207,7 +208,7 @@ def sol_attn2_fp8_rows(q8_rows, row0, k8_bh, v8_bh, mask_row, counts, kg, vg, qb
     return out
 
 
-def sol_attn2_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None):
+def sol_attn2_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, mask_override=None):
     """FP8 + ExpCast Sol-Attn2 forward (R21).  Same return convention as :func:`sol_attn_fp8`."""
     B, N, H, _ = q.shape
     Nb = orc.num_blocks(N)
@@ -223,8 +224,8 @@ def sol_attn2_fp8(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 
             qbar_anchor = orc.block_means(q_bh, orc.ANCHOR)
             q8, k8 = quantize_blocks(q_bh), quantize_blocks(k_bh)
             v8 = quantize(v_bh)[0]
+            use = r["mask"] if mask_override is None else np.asarray(mask_override[b, h], dtype=bool)
             for i in (range(Nb) if qblocks is None else qblocks):
                 lo, hi = orc.block_range(i, N)
-                out[b, lo:hi, h] = sol_attn2_fp8_rows(q8[lo:hi], lo, k8, v8, r["mask"][i], counts, kg, vg,
-                                                      qbar_anchor)
+                out[b, lo:hi, h] = sol_attn2_fp8_rows(q8[lo:hi], lo, k8, v8, use[i], counts, kg, vg, qbar_anchor)
     return dict(out=out, mask=masks)

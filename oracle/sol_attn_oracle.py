@@ -261,12 +261,16 @@ def _row_subset(N, qblocks):
 
 
 def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None,
-             thresh_type: str = "exact", extra_sinks=()):
+             thresh_type: str = "exact", extra_sinks=(), mask_override=None):
     """Sol-Attn forward. Returns dict with ``out`` (FP64 [B, N, H, 128]; NaN for rows not computed),
     ``mask`` [B, H, Nb, Nb], ``shat``, ``thresh``.
 
     ``qblocks``: optional iterable of query-block indices to evaluate (all heads); ``heads``:
     optional iterable of (b, h) pairs.  Summaries and thresholds are always computed in full.
+    ``mask_override``: optional bool [B, H, Nb, Nb] exact sets to evaluate the outputs with instead
+    of this routing's (the parity rule for pairs whose proxy lies within the margin of its
+    threshold, where a kernel's rounding may decide the other way); ``mask`` still reports the
+    oracle's own routing.
     """
     B, N, H, _ = q.shape
     Nb = num_blocks(N)
@@ -281,9 +285,10 @@ def sol_attn(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qb
         r = _routing_for_head(q_bh, k_bh, tau, sink, thresh_type)
         Vhat = block_sums(v_bh)
         masks[b, h], shats[b, h], threshs[b, h] = r["mask"], r["shat"], r["thresh"]
+        use = r["mask"] if mask_override is None else np.asarray(mask_override[b, h], dtype=bool)
         for i in _row_subset(N, qblocks):
             lo, hi = block_range(i, N)
-            out[b, lo:hi, h] = sol_attn_rows(q_bh[lo:hi], k_bh, v_bh, r["mask"][i], r["Kbar"], Vhat, r["counts"])
+            out[b, lo:hi, h] = sol_attn_rows(q_bh[lo:hi], k_bh, v_bh, use[i], r["Kbar"], Vhat, r["counts"])
     return dict(out=out, mask=masks, shat=shats, thresh=threshs)
 
 
@@ -364,10 +369,11 @@ def sol_attn2_rows(q_rows, row0, k_bh, v_bh, mask_row, counts, kg, vg, qbar_anch
 
 
 def sol_attn2(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, qblocks=None, heads=None,
-              extra_sinks=()):
+              extra_sinks=(), mask_override=None):
     """Sol-Attn2 forward (complementary tail). Same return convention as :func:`sol_attn`, plus
     ``group_counts`` [B, H, Nb, 2]: n_g of the two key groups of every block (group 1 = the keys
-    whose projection on the direction lies strictly above the block mean's)."""
+    whose projection on the direction lies strictly above the block mean's).  ``mask_override`` as in
+    :func:`sol_attn`."""
     B, N, H, _ = q.shape
     Nb = num_blocks(N)
     sink = sink_block_flags(N, sink_start, sink_tokens, extra_sinks)
@@ -382,10 +388,10 @@ def sol_attn2(q, k, v, tau: float, sink_start: int = -1, sink_tokens: int = 0, q
         counts, kg, vg = key_groups(k_bh, v_bh, group_direction(q_bh, k_bh))
         group_counts[b, h] = counts
         qbar_anchor = block_means(q_bh, ANCHOR)
+        use = r["mask"] if mask_override is None else np.asarray(mask_override[b, h], dtype=bool)
         for i in _row_subset(N, qblocks):
             lo, hi = block_range(i, N)
-            out[b, lo:hi, h] = sol_attn2_rows(q_bh[lo:hi], lo, k_bh, v_bh, r["mask"][i], counts, kg, vg,
-                                              qbar_anchor)
+            out[b, lo:hi, h] = sol_attn2_rows(q_bh[lo:hi], lo, k_bh, v_bh, use[i], counts, kg, vg, qbar_anchor)
     return dict(out=out, mask=masks, group_counts=group_counts)
 
 

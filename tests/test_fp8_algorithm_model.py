@@ -81,7 +81,28 @@ class _Half:
         self.l = F(self.l + p.sum(dtype=F))
 
 
-def _model_head(q, k, v, tau, sol2, sink_start=-1, sink_tokens=0):
+def _bf16(x):
+    return torch.tensor(np.asarray(x, F)).to(torch.bfloat16).float().numpy()
+
+
+def _tail_model(qbar_a, counts, tk, tv):
+    """The tail kernel's arithmetic (sol2_tail_tc.cu): BF16 anchor and group means as the product
+    operands, FP32 scores, base-2 weights against the row maximum, the FP32 weight sum as Z, BF16
+    weights in the numerators of mu and nu.  Returns (log Z, mu, nu) like orc.anchor_tail."""
+    if len(counts) == 0:
+        return -np.inf, np.zeros(128), np.zeros(128)
+    kh, vh = _bf16(tk), _bf16(tv)
+    y = ((kh @ _bf16(qbar_a)).astype(F) * F(SCALE * LOG2E) + np.log2(counts.astype(F))).astype(F)
+    mx = F(y.max())
+    p = np.exp2(y - mx).astype(F)
+    lsum = p.sum(dtype=F)
+    pb = _bf16(p)
+    return (float(mx) + math.log2(float(lsum))) * math.log(2.0), (pb @ kh) / lsum, (pb @ vh) / lsum
+
+
+def _model_head(q, k, v, tau, sol2, sink_start=-1, sink_tokens=0, bf16_tail=False):
+    """bf16_tail: the Sol-Attn2 tail as the GPU's tail kernel computes it (BF16 operands); otherwise
+    the reference's FP64 tail, so that the comparison with the reference isolates the FP8 path."""
     N = q.shape[0]
     Nb = orc.num_blocks(N)
     r = orc._routing_for_head(q, k, tau, orc.sink_block_flags(N, sink_start, sink_tokens))
@@ -137,7 +158,8 @@ def _model_head(q, k, v, tau, sol2, sink_start=-1, sink_tokens=0):
                 un = np.nonzero(~mask[qi])[0]
                 tc, tk, tv = gcounts[un].reshape(-1), kg[un].reshape(-1, 128), vg[un].reshape(-1, 128)
                 keep = tc > 0
-                logz, mu, nu = orc.anchor_tail(qanchor[tok // orc.ANCHOR], tc[keep], tk[keep], tv[keep])
+                tail_fn = _tail_model if bf16_tail else orc.anchor_tail
+                logz, mu, nu = tail_fn(qanchor[tok // orc.ANCHOR], tc[keep], tk[keep], tv[keep])
                 if np.isfinite(logz):
                     delta = float(SCALE) * ((q8[tok] * sq[qi] - qanchor[tok // orc.ANCHOR]) @ mu)
                     tail = 2.0 ** ((logz + delta) / math.log(2.0) - M)

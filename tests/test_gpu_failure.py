@@ -7,7 +7,7 @@ import torch
 from block_sparse_attention_sum_b200 import sol_attn as sa
 from block_sparse_attention_sum_b200.inputs import iid_qkv
 from oracle import sol_attn_oracle as orc
-from tests.parity import check_mask, compare_outputs
+from tests.parity import check_mask, compare_outputs, with_gpu_mask
 
 pytestmark = pytest.mark.gpu
 
@@ -26,5 +26,6 @@ def test_bounded_wait_runs_out_and_is_reported():
     assert sa.get_device_status() == 0
     ref = orc.sol_attn(q, k, v, 1.0)
     mask, _ = sa.debug_route(q.cuda(), k.cuda(), 1.0)
-    skip = check_mask(mask.cpu().numpy(), ref)
-    compare_outputs(out.float().cpu().numpy(), ref["out"], 700, skip_rows=skip)
+    gm = mask.cpu().numpy()
+    skip = check_mask(gm, ref)
+    compare_outputs(out.float().cpu().numpy(), with_gpu_mask(orc.sol_attn, (q, k, v, 1.0), gm, skip, ref["out"]), 700)

@@ -16,7 +16,7 @@ from block_sparse_attention_sum_b200 import sol_attn as sa
 from block_sparse_attention_sum_b200.inputs import iid_qkv
 from block_sparse_attention_sum_b200.workloads import WORKLOADS
 from oracle import sol_attn_oracle as orc
-from tests.parity import check_mask, compare_outputs
+from tests.parity import check_mask, compare_outputs, with_gpu_mask
 
 pytestmark = pytest.mark.gpu
 
@@ -63,8 +63,9 @@ def test_small_and_ragged(case, entry):
     gmask, gthr = sa.debug_route(qd, kd, tau, ss, st)
     full = orc.routing(q, k, tau, ss, st)
     ref.update(shat=full["shat"], thresh=full["thresh"])
-    skip = check_mask(gmask.cpu().numpy(), ref, orc.sink_block_flags(N, ss, st))
-    compare_outputs(gout, ref["out"], N, skip_rows=skip)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref, orc.sink_block_flags(N, ss, st))
+    compare_outputs(gout, with_gpu_mask(getattr(orc, entry), (q, k, v, tau, ss, st), gm, skip, ref["out"]), N)
 
 
 @pytest.mark.parametrize("name", ["tiny", "wan"])
@@ -78,10 +79,12 @@ def test_named_workloads_in_full(name, entry):
     ref.update(shat=full["shat"], thresh=full["thresh"])
     gout, (qd, kd, _) = _run(entry, q, k, v, tau, w.sink_start, w.sink_tokens)
     gmask, gthr = sa.debug_route(qd, kd, tau, w.sink_start, w.sink_tokens)
-    skip = check_mask(gmask.cpu().numpy(), ref)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref)
     assert skip.mean() <= 0.01
     np.testing.assert_allclose(gthr.cpu().numpy(), full["thresh"], rtol=1e-5, atol=2e-6)
-    compare_outputs(gout, ref["out"], w.N, skip_rows=skip)
+    args = (q, k, v, tau, w.sink_start, w.sink_tokens)
+    compare_outputs(gout, with_gpu_mask(getattr(orc, entry), args, gm, skip, ref["out"]), w.N)
 
 
 LARGE = ["s32k_80", "s32k_85", "s32k_90", "s64k", "s128k", "sol2_64k"]
@@ -108,7 +111,10 @@ def test_large_workloads_sampled(name):
     assert exact == int(gm.sum()) and total == gm.size
     assert abs((1 - exact / total) - w.target_sparsity) < 0.01
     np.testing.assert_allclose(gthr.cpu().numpy(), ref["thresh"], rtol=1e-5, atol=2e-6)
-    compare_outputs(gout, ref["out"], w.N, skip_rows=skip)
+    # rows of sampled query blocks whose masks differ: the oracle with the GPU's exact sets
+    skip &= np.isin(np.arange(Nb), sample)[None, None, :]
+    args = (q, k, v, tau, w.sink_start, w.sink_tokens)
+    compare_outputs(gout, with_gpu_mask(fn, args, gm, skip, ref["out"]), w.N)
 
 
 def test_repeated_calls_are_bitwise_identical():
@@ -167,9 +173,12 @@ def test_diagonal_threshold_estimator(name):
     torch.cuda.synchronize()
     assert sa.get_device_status() == 0
     gmask, gthr = sa.debug_route(qd, kd, tau, w.sink_start, w.sink_tokens, thresh_type="diag")
-    skip = check_mask(gmask.cpu().numpy(), ref)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref)
     np.testing.assert_allclose(gthr.cpu().numpy(), full["thresh"], rtol=1e-5, atol=2e-6)
-    compare_outputs(out.float().cpu().numpy(), ref["out"], w.N, skip_rows=skip)
+    args = (q, k, v, tau, w.sink_start, w.sink_tokens)
+    compare_outputs(out.float().cpu().numpy(), with_gpu_mask(orc.sol_attn, args, gm, skip, ref["out"], thresh_type="diag"),
+                    w.N)
     exact = orc.routing(q, k, tau, w.sink_start, w.sink_tokens)
     assert not np.array_equal(exact["mask"], full["mask"])   # the estimator changes the routing
 
@@ -192,8 +201,10 @@ def test_extra_sink_ranges(entry):
     gmask, _ = sa.debug_route(qd, kd, tau, 0, 100, extra_sinks=extra)
     flags = orc.sink_block_flags(N, 0, 100, extra)
     assert flags.sum() >= 7
-    skip = check_mask(gmask.cpu().numpy(), ref, sink_flags=flags)
-    compare_outputs(out.float().cpu().numpy(), ref["out"], N, skip_rows=skip)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref, sink_flags=flags)
+    compare_outputs(out.float().cpu().numpy(),
+                    with_gpu_mask(fn, (q, k, v, tau, 0, 100), gm, skip, ref["out"], extra_sinks=extra), N)
 
 
 @pytest.mark.parametrize("rows", [(70, 131), (0, 64), (-1, 40), (1500, 10_000)])
@@ -231,8 +242,10 @@ def test_split_kv(case, kv_splits):
     assert sa.get_device_status() == 0
     assert sa.last_launch_count() == 8   # routing (6) + fused kernel + combine
     gmask, _ = sa.debug_route(qd, kd, tau, ss, st)
-    skip = check_mask(gmask.cpu().numpy(), ref)
-    compare_outputs(out.float().cpu().numpy(), ref["out"], N, skip_rows=skip)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref)
+    compare_outputs(out.float().cpu().numpy(), with_gpu_mask(orc.sol_attn, (q, k, v, tau, ss, st), gm, skip, ref["out"]),
+                    N)
     one = sa.sol_attn_fwd(qd, kd, vd, tau, ss, st)
     torch.cuda.synchronize()
     assert (out.float() - one.float()).abs().max().item() <= 1.6e-2
@@ -264,5 +277,6 @@ def test_varlen_packed_batch():
         qs, ks, vs = q[:, sl], k[:, sl], v[:, sl]
         ref = orc.sol_attn(qs, ks, vs, tau, 0, 32)
         gmask, _ = sa.debug_route(qs.cuda(), ks.cuda(), tau, 0, 32)
-        skip = check_mask(gmask.cpu().numpy(), ref)
-        compare_outputs(got[None, sl], ref["out"], n, skip_rows=skip)
+        gm = gmask.cpu().numpy()
+        skip = check_mask(gm, ref)
+        compare_outputs(got[None, sl], with_gpu_mask(orc.sol_attn, (qs, ks, vs, tau, 0, 32), gm, skip, ref["out"]), n)

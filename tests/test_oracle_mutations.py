@@ -156,6 +156,13 @@ def _sol_attn2_per_query_block_direction(q, k, v, tau, sink_start=-1, sink_token
     return dict(out=out, mask=masks, group_counts=group_counts)
 
 
+_orig_sol_attn = orc.sol_attn
+
+
+def _override_ignored(q, k, v, tau, *args, mask_override=None, **kw):
+    return _orig_sol_attn(q, k, v, tau, *args, **kw)
+
+
 CASES = [
     ("block_sums", _value_means_not_sums,
      lambda: pins.test_identical_unselected_keys_make_the_approximation_exact(448, "sol_attn")),
@@ -182,6 +189,7 @@ CASES = [
     ("key_groups", _ties_upper, pins.test_hand_expanded_sol_attn2_split_direction),
     ("key_groups", _groups_median_split, pins.test_hand_expanded_sol_attn2_split_direction),
     ("sol_attn2", _sol_attn2_per_query_block_direction, pins.test_hand_expanded_sol_attn2_split_direction),
+    ("sol_attn", _override_ignored, lambda: pins.test_mask_override_evaluates_the_given_exact_sets("sol_attn")),
 ]
 
 

@@ -295,6 +295,23 @@ def test_hand_expanded_sol_attn2_split_direction():
             np.testing.assert_allclose(r["out"][0, row, 0], expect, rtol=1e-11, atol=1e-14)
 
 
+# ------------------------------------------------------------------------- mask override (parity)
+
+@pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
+def test_mask_override_evaluates_the_given_exact_sets(entry):
+    """The override used by the GPU parity rule: the oracle's own mask reproduces its result, and an
+    all-exact mask gives textbook softmax attention (Eq. (2) with every block selected), whatever
+    the routing decided."""
+    q, k, v = rand_qkv(1, 300, 2, seed=41)
+    fn = getattr(orc, entry)
+    r = fn(q, k, v, 1.0)
+    assert not r["mask"].all()
+    np.testing.assert_array_equal(fn(q, k, v, 1.0, mask_override=r["mask"])["out"], r["out"])
+    dense = fn(q, k, v, 1.0, mask_override=np.ones_like(r["mask"]))
+    np.testing.assert_allclose(dense["out"], dense_attention(q, k, v), rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(dense["mask"], r["mask"])      # the routing is still reported
+
+
 # ---------------------------------------------------------------------------- Sol-Attn2 groups
 
 def test_group_counts_preserve_block_mass():

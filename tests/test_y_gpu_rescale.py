@@ -22,7 +22,7 @@ import torch
 from block_sparse_attention_sum_b200 import sol_attn as sa
 from block_sparse_attention_sum_b200.inputs import iid_qkv
 from oracle import sol_attn_oracle as orc
-from tests.parity import check_mask, compare_outputs
+from tests.parity import check_mask, compare_outputs, model_rows_with_agreeing_masks, with_gpu_mask
 
 pytestmark = pytest.mark.gpu
 
@@ -49,8 +49,9 @@ def test_bf16_running_max_jump_matches_the_reference(entry, tau):
     full = orc.routing(q, k, tau)
     ref.update(shat=full["shat"], thresh=full["thresh"])
     gmask, _ = sa.debug_route(qd, kd, tau)
-    skip = check_mask(gmask.cpu().numpy(), ref)
-    compare_outputs(out.float().cpu().numpy(), ref["out"], N, skip_rows=skip)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref)
+    compare_outputs(out.float().cpu().numpy(), with_gpu_mask(getattr(orc, entry), (q, k, v, tau), gm, skip, ref["out"]), N)
 
 
 @pytest.mark.parametrize("tau", [-10.0, 1.0], ids=["dense", "tau1"])
@@ -63,9 +64,7 @@ def test_fp8_pivot_jump_matches_the_fp32_model(entry, tau):
     out = (sa.sol_attn_fwd_fp8 if entry == "sol_attn" else sa.sol_attn2_fwd_fp8)(qd, kd, vd, tau)
     torch.cuda.synchronize()
     assert sa.get_device_status() == 0
-    from tests.test_zzz_gpu_fp8 import model_rows_with_agreeing_masks
-
-    model = _model_head(*(orc.head_slice(t, 0, 0) for t in (q, k, v)), tau, entry == "sol_attn2")
+    model = _model_head(*(orc.head_slice(t, 0, 0) for t in (q, k, v)), tau, entry == "sol_attn2", bf16_tail=True)
     model = torch.tensor(model).to(torch.bfloat16).float().numpy()
     rows = model_rows_with_agreeing_masks(qd, kd, q, k, tau)
     d = out.float().cpu().numpy()[0, rows, 0] - model[rows]
