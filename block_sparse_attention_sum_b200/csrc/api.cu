@@ -295,7 +295,10 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   if (rc) return rc;
   Work ww = w;
   ww.stats = d.stats;
-  launch_summary(q, k, v, s, ww, anchors, st);
+  if (anchors)
+    launch_sol2_summaries(q, k, v, s, ww, st);   // Sol-Attn2: the key groups come with the key means
+  else
+    launch_summary(q, k, v, s, ww, false, st);
   launch_kstats(s, ww, st);
   launch_thresh(s, ww, tau, diag, st);
   CUtensorMap rmaps[4];
@@ -304,7 +307,7 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
     return rc;
   cudaError_t e = launch_route_tc(rmaps, s, ww, sinks, d.status, st);
   if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "routing launch: %s", cudaGetErrorString(e));
-  *launches += 6;
+  *launches += anchors ? 8 : 6;
   d.last_total_pairs = (long long)s.BH * s.Nb * s.Nb;
   return check_launch("routing kernels");
 }
@@ -393,10 +396,9 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
     if ((rc = encode_rows(&tmaps[0], w.qanchor_h, s.Na, s)) || (rc = encode_rows(&tmaps[1], w.gk_h, 2 * s.Nb, s)) ||
         (rc = encode_rows(&tmaps[2], w.gv_h, 2 * s.Nb, s)))
       return rc;
-    launch_groups(qh, kh, vh, s, w, st);
     cudaError_t te = launch_tail_tc(tmaps, s, w, d->status, st);
     if (te != cudaSuccess) return fail(SOL_ERR_LAUNCH, "Sol-Attn2 tail launch: %s", cudaGetErrorString(te));
-    launches += 3;
+    launches += 1;
     if ((rc = check_launch("Sol-Attn2 tail kernels"))) return rc;
   }
   if (fp8) {

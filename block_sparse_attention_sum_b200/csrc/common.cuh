@@ -88,9 +88,10 @@ void launch_expand_mask(const Shape& s, const Work& w, unsigned char* mask_out, 
 // Sets every valid bit of the bitmask rows of query blocks qb_lo .. qb_hi (all heads).
 void launch_dense_mask(const Shape& s, const Work& w, int qb_lo, int qb_hi, cudaStream_t st);
 
-// Sol-Attn2 prep (sol2_tail.cu)
-void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                   const Work& w, cudaStream_t st);
+// Sol-Attn2 summaries (sol2_tail.cu), in place of launch_summary: query and anchor means, the mean
+// query, then key means and the two key groups of every block (three launches).
+void launch_sol2_summaries(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
+                           const Work& w, cudaStream_t st);
 // Sol-Attn2 tail statistics on the tensor cores (sol2_tail_tc.cu); maps = anchor means, group key
 // means, group value means (BF16, 3-D, box 64 x 128 x 1, 128-byte swizzle).
 cudaError_t launch_tail_tc(const void* maps, const Shape& s, const Work& w, int* status, cudaStream_t st);

@@ -4,8 +4,9 @@
 // complementary approximation": each unselected key block is split into two content groups by its
 // keys' projection on the mean-query direction.  The direction is the mean of all queries of the
 // (batch, head), so the groups do not depend on the query and are built once here, for every key
-// block; the per-anchor tail statistics over them are computed on the tensor cores
-// (sol2_tail_tc.cu).
+// block, in the same pass over K and V that computes the block means: a query pass (query and
+// anchor means), the direction, then the key / value pass.  The per-anchor tail statistics over
+// the groups are computed on the tensor cores (sol2_tail_tc.cu).
 #include <cfloat>
 #include <cmath>
 
@@ -39,12 +40,94 @@ __global__ void __launch_bounds__(1024) qdir_kernel(Shape s, Work w) {
   }
 }
 
-// Two groups per key block: group 1 = keys with k.u > Kbar_j.u, group 0 = the rest (FP32 decision).
-// One CTA per (key block j, b, h), the block-summary kernel's access pattern: 16 threads cover a
-// 256-byte row with 16-byte loads, 16 row groups cover the block, all loads issued up front.
-__global__ void __launch_bounds__(256) groups_kernel(const __nv_bfloat16* __restrict__ k,
-                                                     const __nv_bfloat16* __restrict__ v, Shape s, Work w) {
+// Query pass of the Sol-Attn2 summaries: Qbar (FP32 and the BF16 hi / lo split of the routing
+// product) and the two 32-token anchor means of every block.  One CTA per (query block j, b, h)
+// with summary_kernel's thread mapping and summation order, so Qbar is bit-identical to the
+// Sol-Attn path's.
+__global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __restrict__ q, Shape s, Work w) {
+  __shared__ float red[8][2][kHeadDim];
+  const int j = blockIdx.x, b = blockIdx.y / s.H, h = blockIdx.y % s.H;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c16 = tid & 15, rg = tid >> 4;
+  const int t0 = j * kBlock;
+  const int n = min(kBlock, s.N - t0);
+  const int nlo = min(n, kAnchor), nhi = n - nlo;
+  float qlo[8], qhi[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) qlo[e] = qhi[e] = 0.f;
+  uint4 rq[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int r = rg + 16 * m;
+    rq[m] = r < n ? __ldg(reinterpret_cast<const uint4*>(q + ((size_t)(b * (size_t)s.N + t0 + r) * s.H + h) * kHeadDim +
+                                                        8 * c16))
+                  : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const __nv_bfloat162* pq = reinterpret_cast<const __nv_bfloat162*>(&rq[m]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fq = __bfloat1622float2(pq[e]);
+      if (m < 2) {
+        qlo[2 * e] += fq.x;
+        qlo[2 * e + 1] += fq.y;
+      } else {
+        qhi[2 * e] += fq.x;
+        qhi[2 * e + 1] += fq.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    qlo[e] += __shfl_xor_sync(0xffffffffu, qlo[e], 16);
+    qhi[e] += __shfl_xor_sync(0xffffffffu, qhi[e], 16);
+  }
+  if (lane < 16) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      red[warp][0][8 * c16 + e] = qlo[e];
+      red[warp][1][8 * c16 + e] = qhi[e];
+    }
+  }
+  __syncthreads();
+  if (tid < kHeadDim) {
+    const int c = tid;
+    float sqlo = 0.f, sqhi = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) {
+      sqlo += red[ww][0][c];
+      sqhi += red[ww][1][c];
+    }
+    const size_t bh = (size_t)b * s.H + h;
+    const size_t o = (bh * s.Nb + j) * kHeadDim + c;
+    const float qb = (sqlo + sqhi) / (float)n;
+    w.qbar[o] = qb;
+    const __nv_bfloat16 qh = __float2bfloat16_rn(qb);
+    w.qbar_hi[o] = qh;
+    w.qbar_lo[o] = __float2bfloat16_rn(qb - __bfloat162float(qh));
+    const size_t a0 = (bh * s.Na + 2 * (size_t)j) * kHeadDim + c;
+    const float alo = sqlo / (float)nlo;
+    w.qanchor[a0] = alo;
+    w.qanchor_h[a0] = __float2bfloat16_rn(alo);
+    if (nhi > 0) {
+      const float ahi = sqhi / (float)nhi;
+      w.qanchor[a0 + kHeadDim] = ahi;
+      w.qanchor_h[a0 + kHeadDim] = __float2bfloat16_rn(ahi);
+    }
+  }
+}
+
+// Key / value pass of the Sol-Attn2 summaries, after the mean query u is known: Kbar (FP32 and the
+// BF16 hi / lo split of the routing product; summary_kernel's summation order, so bit-identical)
+// and the block's two key groups: group 1 = keys with k.u > Kbar_j.u, group 0 = the rest (FP32
+// decision), their sizes, key means and value means.  K and V are read once, kept in registers
+// between the block-mean reduction and the group split.  One CTA per (key block j, b, h): 16
+// threads cover a 256-byte row with 16-byte loads, 16 row groups cover the block.
+__global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloat16* __restrict__ k,
+                                                                const __nv_bfloat16* __restrict__ v, Shape s, Work w) {
   __shared__ float red[8][4][kHeadDim];
+  __shared__ float kbar_s[kHeadDim];
   __shared__ int n1_s;
   const int j = blockIdx.x, bh = blockIdx.y, b = bh / s.H, h = bh % s.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -64,15 +147,51 @@ __global__ void __launch_bounds__(256) groups_kernel(const __nv_bfloat16* __rest
       rk[m] = rv[m] = make_uint4(0, 0, 0, 0);
     }
   }
-  // the cut Kbar_j . u, reduced over the 16 lanes of a row group (each holds 8 channels)
+  // ---- block mean of the keys
+  {
+    float ks[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ks[e] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const __nv_bfloat162* pk = reinterpret_cast<const __nv_bfloat162*>(&rk[m]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fk = __bfloat1622float2(pk[e]);
+        ks[2 * e] += fk.x;
+        ks[2 * e + 1] += fk.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], 16);
+    if (lane < 16) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[warp][0][8 * c16 + e] = ks[e];
+    }
+    __syncthreads();
+    if (tid < kHeadDim) {
+      const int c = tid;
+      float sk = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww) sk += red[ww][0][c];
+      const size_t o = ((size_t)bh * s.Nb + j) * kHeadDim + c;
+      const float kb = sk / (float)n;
+      w.kbar[o] = kb;
+      const __nv_bfloat16 kh = __float2bfloat16_rn(kb);
+      w.kbar_h[o] = kh;
+      w.kbar_lo[o] = __float2bfloat16_rn(kb - __bfloat162float(kh));
+      kbar_s[c] = kb;
+    }
+    __syncthreads();
+  }
+  // ---- the two groups: the cut Kbar_j . u, reduced over the 16 lanes of a row group
   const float* u = w.qdir + (size_t)bh * kHeadDim + 8 * c16;
-  const float* kb = w.kbar + ((size_t)bh * s.Nb + j) * kHeadDim + 8 * c16;
   float uu[8];
   float cut = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     uu[e] = u[e];
-    cut = fmaf(kb[e], uu[e], cut);
+    cut = fmaf(kbar_s[8 * c16 + e], uu[e], cut);
   }
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) cut += __shfl_xor_sync(0xffffffffu, cut, o);
@@ -118,7 +237,6 @@ __global__ void __launch_bounds__(256) groups_kernel(const __nv_bfloat16* __rest
     v0[e] += __shfl_xor_sync(0xffffffffu, v0[e], 16);
     v1[e] += __shfl_xor_sync(0xffffffffu, v1[e], 16);
   }
-  __syncthreads();   // n1_s initialised
   if (c16 == 0 && n1) atomicAdd(&n1_s, n1);
   if (lane < 16) {
 #pragma unroll
@@ -153,11 +271,11 @@ __global__ void __launch_bounds__(256) groups_kernel(const __nv_bfloat16* __rest
   }
 }
 
-void launch_groups(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                   const Work& w, cudaStream_t st) {
-  (void)q;
+void launch_sol2_summaries(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
+                           const Work& w, cudaStream_t st) {
+  summary_q_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, s, w);
   qdir_kernel<<<s.BH, 8 * kHeadDim, 0, st>>>(s, w);
-  groups_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(k, v, s, w);
+  summary_kv_groups_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(k, v, s, w);
 }
 
 }  // namespace sol
