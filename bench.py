@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -51,7 +52,13 @@ def parse_args():
                     help="attention products in BF16 (default) or E4M3 with ExpCast weights (sol_attn*_fwd_fp8)")
     ap.add_argument("--no-fp8-leg", action="store_true",
                     help="skip the FP8 companion measurement that a one-GPU BF16 run adds to its line")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the other workloads of the metric's range that a one-GPU s64k run adds to its line")
     return ap.parse_args()
+
+
+# the rest of the metric's range (32K-128K tokens, 32 heads), measured after the headline workload
+LEG_WORKLOADS = ["sol2_64k", "s32k_80", "s32k_85", "s32k_90", "s128k"]
 
 
 def rank_seed(workload, rank: int) -> int:
@@ -269,6 +276,82 @@ def fp8_leg(sa, w, q, k, v, out_bf16, tau, stream, flops_step, peaks, steps):
         return {"error": f"{type(e).__name__}: {e}"[:300]}
 
 
+def workload_leg(sa, w, inputs, dev, stream, steps, peaks):
+    """One more workload timed like the headline one (inputs resident in HBM, CUDA events around
+    ``steps`` calls after 3 warm-up calls, the fused kernel's own time from the library's events,
+    SM clocks sampled during the timed calls).  Any failure is reported in the object, never raised."""
+    import torch
+
+    try:
+        q, k, v = inputs
+        out = torch.empty_like(q)
+        tau = w.resolved_tau()
+        fn = sa.sol_attn_fwd if w.entry == "sol_attn" else sa.sol_attn2_fwd
+
+        def step():
+            fn(q, k, v, tau, w.sink_start, w.sink_tokens, out=out, stream=stream)
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        if sa.get_device_status() != 0:
+            return {"error": "device status reports a timed-out wait after the warm-up"}
+        exact, total, min_row, max_row = sa.last_stats()
+        launches = sa.last_launch_count()
+        # at least ~0.4 s of timed calls, so that the clock sampler (every 100 ms) sees the leg
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        steps = int(min(200, max(steps, math.ceil(400.0 / max(a.elapsed_time(b), 1e-3)))))
+        clocks = ClockSampler(dev.index or 0)
+        time.sleep(0.3)   # the sampler's first reading
+        sa.set_kernel_timing(True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        clock_info = clocks.stop()
+        kernel_ms = sa.kernel_ms_sum(steps) / steps
+        sa.set_kernel_timing(False)
+        if sa.get_device_status() != 0:
+            return {"error": "device status reports a timed-out wait in the timed calls"}
+        ms = a.elapsed_time(b) / steps
+        flops, exact_flops = effective_flops(w.B, w.N, w.H, exact, total)
+        if w.entry == "sol_attn2":
+            flops = sol2_flops(w.B, w.N, w.H, exact, total)
+        burst = float(peaks["bf16_tflops"])
+        sust = float(peaks.get("bf16_tflops_sustained", burst))
+        value = flops / (ms * 1e-3) / 1e12
+        kernel_tflops = flops / (kernel_ms * 1e-3) / 1e12
+        kname = "attn_fwd_kernel" + ("<false>" if w.entry == "sol_attn" else "<true>")
+        return {"entry": fn.__name__, "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d=128", "tau": tau,
+                "sink": [w.sink_start, w.sink_tokens], "target_sparsity": w.target_sparsity,
+                "realised_sparsity": 1.0 - exact / total, "min_row": min_row, "max_row": max_row,
+                "steps": steps, "warmup": 3, "ms_per_step": ms, "value": value, "unit": "TFLOP/s",
+                "frac_of_peak": value / burst, "frac_of_sustained_peak": value / sust,
+                "exact_only_tflops": exact_flops / (ms * 1e-3) / 1e12,
+                "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": burst, "unit": "TFLOP/s",
+                             "frac": kernel_tflops / burst, "kernel": kname + " (fused attention)",
+                             "kernel_ms": kernel_ms, "peak_kind": f"bf16 dense burst ({peaks['source']})"},
+                "gpu_launches": launches * steps, "clocks": clock_info}
+    except Exception as e:   # reported, so that the headline line is printed whatever happens here
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
+def sol2_flops(B, N, H, exact_pairs, total_pairs, d=128):
+    """Sol-Attn2 effective FLOPs: the exact pairs as for Sol-Attn; the tail costs 12 d per
+    (anchor, unselected block) pair (S against the two groups, then [kbar_g | vbar_g]) and the
+    first-order correction 2 d per query token."""
+    Nb = (N + 63) // 64
+    exact_flops = 4.0 * d * (N / Nb) ** 2 * exact_pairs
+    anchors_per_block = (N / Nb) / 32.0
+    return exact_flops + 12.0 * d * anchors_per_block * (total_pairs - exact_pairs) + 2.0 * d * B * H * N
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -347,7 +430,7 @@ def main():
         step()
     torch.cuda.synchronize()
     assert sa.get_device_status() == 0, "device status after warm-up"
-    exact, total, _, _ = sa.last_stats()
+    exact, total, min_row, max_row = sa.last_stats()
     launches_per_step = sa.last_launch_count()
 
     def barrier():
@@ -356,6 +439,7 @@ def main():
 
     # ---- timed region: inputs resident in HBM
     clocks = ClockSampler(local_rank)
+    time.sleep(0.3)   # the sampler's first reading
     sa.set_kernel_timing(True)
     barrier()
     torch.cuda.synchronize()
@@ -375,6 +459,8 @@ def main():
     elapsed_ms, kernel_ms = max_over_ranks([elapsed_ms, kernel_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
     flops_step, exact_flops_step = effective_flops(w.B, w.N, w.H, exact, total)
+    if w.entry == "sol_attn2":
+        flops_step = sol2_flops(w.B, w.N, w.H, exact, total)
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
     sp = 1.0 - exact / total
     gmask, _ = sa.debug_route(q, k, tau, w.sink_start, w.sink_tokens)
@@ -432,6 +518,7 @@ def main():
                        "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "tau": tau,
                        "target_sparsity": w.target_sparsity, "realised_sparsity": sp,
                        "union_tile_useful_fraction": union_frac, "kv_splits": args.kv_splits,
+                       "min_row": min_row, "max_row": max_row,
                        "precision": args.precision,
                        "parallelism": f"independent replicas x{world} (head/batch sharding, no exchange)",
                        "l2": "inputs 1.6 GB per rank > 126 MB L2; no flush"},
@@ -443,17 +530,36 @@ def main():
 
     if world == 1 and not fp8 and not args.no_fp8_leg:
         line["fp8"] = fp8_leg(sa, w, q, k, v, out, tau, stream, flops_step, peaks, args.steps)
+    if world == 1 and not fp8 and not args.no_legs and w.name == "s64k" and args.kv_splits == 1:
+        def inputs_key(x):   # workloads that differ only in tau target or sink share their inputs
+            return x.input_key().split("@")[0].split("+")[0]
+
+        legs, cache = {}, {inputs_key(w): (q, k, v)}
+        for name in LEG_WORKLOADS:
+            lw = WORKLOADS[name]
+            key = inputs_key(lw)
+            if key not in cache:
+                cache.clear()
+                torch.cuda.empty_cache()
+                cache[key] = tuple(t.to(dev) for t in lw.make_inputs("cpu"))
+            legs[name] = workload_leg(sa, lw, cache[key], dev, stream, max(5, min(args.steps, 10)), peaks)
+        cache.clear()
+        line["workloads"] = legs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(w, [(0, h) for h in range(args.cpu_sample_heads)], 1 << 30, qh, kh, vh)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world == 1 and "error" in (line.get("fp8") or {}):
-        # the FP8 leg failed after the line was complete: leave without tearing down a CUDA context
-        # that may be unusable, so that the run still ends with status 0 and its line
-        sys.stderr.write(f"fp8 leg: {line['fp8']['error']}\n")
+    leg_errors = [n for n, leg in (line.get("workloads") or {}).items() if "error" in leg]
+    if world == 1 and ("error" in (line.get("fp8") or {}) or leg_errors):
+        # the FP8 leg failed after the line was complete: report it through the exit status, and
+        # leave without tearing down a CUDA context that may be unusable
+        for n in leg_errors:
+            sys.stderr.write(f"{n} leg: {line['workloads'][n]['error']}\n")
+        if "error" in (line.get("fp8") or {}):
+            sys.stderr.write(f"fp8 leg: {line['fp8']['error']}\n")
         sys.stderr.flush()
-        os._exit(0)
+        os._exit(1)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
