@@ -328,7 +328,8 @@ def workload_leg(sa, w, inputs, dev, stream, steps, peaks):
         value = flops / (ms * 1e-3) / 1e12
         kernel_tflops = flops / (kernel_ms * 1e-3) / 1e12
         kname = "attn_fwd_kernel" + ("<false>" if w.entry == "sol_attn" else "<true>")
-        return {"entry": fn.__name__, "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d=128", "tau": tau,
+        sched = scheduler_stats(sa, step)
+        return {"entry": fn.__name__, "scheduler": sched, "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d=128", "tau": tau,
                 "sink": [w.sink_start, w.sink_tokens], "target_sparsity": w.target_sparsity,
                 "realised_sparsity": 1.0 - exact / total, "min_row": min_row, "max_row": max_row,
                 "steps": steps, "warmup": 3, "ms_per_step": ms, "value": value, "unit": "TFLOP/s",
@@ -340,6 +341,31 @@ def workload_leg(sa, w, inputs, dev, stream, steps, peaks):
                 "gpu_launches": launches * steps, "clocks": clock_info}
     except Exception as e:   # reported, so that the headline line is printed whatever happens here
         return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
+def scheduler_stats(sa, step):
+    """One more call with per-CTA timing on: how evenly the hardware's CTA scheduler spreads the
+    fused kernel's work units over the SMs.  tail_frac = (last SM's finish - median SM's finish) /
+    kernel span; busy_frac = time inside CTAs / (span x SMs used)."""
+    import numpy as np
+    import torch
+
+    sa.set_unit_timing(True)
+    try:
+        step()
+        torch.cuda.synchronize()
+        ut = sa.last_unit_times()
+    finally:
+        sa.set_unit_timing(False)
+    start, end, sm = ut[:, 0], ut[:, 1], ut[:, 2]
+    t0 = start.min()
+    span = float(end.max() - t0)
+    sms = np.unique(sm)
+    finish = np.array([end[sm == s].max() - t0 for s in sms], dtype=np.float64)
+    return {"units": int(len(ut)), "sms": int(len(sms)), "span_ms": span / 1e6,
+            "tail_frac": float((finish.max() - np.median(finish)) / span),
+            "busy_frac": float((end - start).sum() / (span * len(sms))),
+            "unit_ms_mean": float((end - start).mean()) / 1e6, "unit_ms_max": float((end - start).max()) / 1e6}
 
 
 def sol2_flops(B, N, H, exact_pairs, total_pairs, d=128):
@@ -456,6 +482,7 @@ def main():
     sa.set_kernel_timing(False)
     assert sa.get_device_status() == 0, "device status after the timed region"
 
+    sched = None if fp8 else scheduler_stats(sa, step)
     elapsed_ms, kernel_ms = max_over_ranks([elapsed_ms, kernel_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
     flops_step, exact_flops_step = effective_flops(w.B, w.N, w.H, exact, total)
@@ -518,7 +545,7 @@ def main():
                        "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "tau": tau,
                        "target_sparsity": w.target_sparsity, "realised_sparsity": sp,
                        "union_tile_useful_fraction": union_frac, "kv_splits": args.kv_splits,
-                       "min_row": min_row, "max_row": max_row,
+                       "min_row": min_row, "max_row": max_row, "scheduler": sched,
                        "precision": args.precision,
                        "parallelism": f"independent replicas x{world} (head/batch sharding, no exchange)",
                        "l2": "inputs 1.6 GB per rank > 126 MB L2; no flush"},

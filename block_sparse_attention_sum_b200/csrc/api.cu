@@ -48,11 +48,15 @@ struct DeviceState {
   cudaStream_t last_stream = nullptr;
   long long last_total_pairs = 0;
   int last_launches = 0;
+  unsigned long long* unit_buf = nullptr;   // per-CTA timing of the fused kernel (when enabled)
+  size_t unit_cap = 0;                      // CTAs the buffer holds
+  int last_units = 0;                       // CTAs of the last timed fused launch
 };
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 bool g_timing = false;
+bool g_unit_timing = false;
 int g_last_device = -1;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -428,6 +432,24 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   p.part_o = part_o;
   p.part_ml = part_ml;
   p.part_rows_bh = rows_bh;
+  if (g_unit_timing && !fp8) {
+    const size_t units = (size_t)s.BH * s.QT * splits;
+    if (d->unit_cap < units) {
+      if (d->unit_buf) {
+        cudaDeviceSynchronize();
+        cudaFree(d->unit_buf);
+      }
+      d->unit_buf = nullptr;
+      d->unit_cap = 0;
+      if (cudaMalloc(&d->unit_buf, units * 3 * sizeof(unsigned long long)) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(SOL_ERR_ALLOC, "unit timing buffer allocation failed");
+      }
+      d->unit_cap = units;
+    }
+    p.unit_times = d->unit_buf;
+    d->last_units = (int)units;
+  }
   const int slot = d->timed_calls % DeviceState::kRing;
   if (g_timing) {
     if (!d->t0[slot] && (cudaEventCreate(&d->t0[slot]) != cudaSuccess || cudaEventCreate(&d->t1[slot]) != cudaSuccess))
@@ -670,6 +692,30 @@ static float kernel_ms_sum_locked(int n) {
     total += ms;
   }
   return (float)total;
+}
+
+int sol_attn_set_unit_timing(int enable) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_unit_timing = enable != 0;
+  return SOL_OK;
+}
+
+int sol_attn_last_unit_times(unsigned long long* host, int max_units, int* units) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!host || !units) return fail(SOL_ERR_NULL, "host and units must be non-NULL");
+  if (g_last_device < 0) return fail(SOL_ERR_LAUNCH, "no call has run yet");
+  DeviceState& d = g_dev[g_last_device];
+  if (!d.unit_buf || d.last_units <= 0) return fail(SOL_ERR_LAUNCH, "no fused launch ran with unit timing enabled");
+  int cur = -1;
+  cudaGetDevice(&cur);
+  cudaSetDevice(g_last_device);
+  const int n = std::min(max_units, d.last_units);
+  cudaError_t e = cudaStreamSynchronize(d.last_stream);
+  if (e == cudaSuccess && n > 0) e = cudaMemcpy(host, d.unit_buf, (size_t)n * 3 * sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+  cudaSetDevice(cur);
+  if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "unit times read failed: %s", cudaGetErrorString(e));
+  *units = d.last_units;
+  return SOL_OK;
 }
 
 float sol_attn_last_kernel_ms(void) {

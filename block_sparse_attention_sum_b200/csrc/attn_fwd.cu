@@ -66,6 +66,7 @@ struct __align__(1024) FwdSmem {
   uint32_t tmem_base;
   int abort;
   int tile_lo, tile_hi;     // this CTA's share [tile_lo, tile_hi) of the unit's tile list
+  unsigned long long t_start;   // %globaltimer at the CTA's start (per-CTA timing only)
 };
 
 // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (checked at run time: a
@@ -165,6 +166,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&sm.mmadone2, 1);
     mbar_init(&sm.lbar, 256);
     sm.abort = 0;
+    if (p.unit_times) sm.t_start = globaltimer();
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -609,38 +611,55 @@ __global__ void __launch_bounds__(384, 1)
       float scale_o = 1.f / l_tot;
       float tail_w = 0.f;
       const float* nu = nullptr;
-      if (kSol2 && row_valid) {
-        const int a = tok / 32;
+      if (kSol2) {
+        // the warp's 32 rows share one anchor: the warp loads mu_a and this warpgroup's half of
+        // nu_a once (coalesced) into the idle K ring (every product is complete here) and reduces
+        // qbar_a . mu_a; each lane then reads them as shared-memory broadcasts, and
+        // delta_i = (q_i . mu_a - qbar_a . mu_a) / sqrt(d)
+        const int a = min(2 * qb0 + (warp & 3), p.Na - 1);
         const size_t abase = (size_t)bh * p.Na + a;
         const float logz = p.tail_logz[abase];
-        if (logz != -INFINITY) {
-          const float* mu = p.tail_mu + abase * 128;
-          const float* qa = p.qanchor + abase * 128;
-          float delta = 0.f;
-          const uint32_t q_row = smem_u32(&sm.q[0][0]) + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll 4
-          for (int c8 = 0; c8 < 16; ++c8) {
-            const uint32_t addr = q_row + (c8 >> 3) * kTileBytes + ((((uint32_t)c8 & 7u) ^ ((uint32_t)r & 7u)) << 4);
-            uint32_t w4[4];
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
-                         : "r"(addr));
+        if (logz != -INFINITY) {   // warp-uniform
+          float* sc_mu = reinterpret_cast<float*>(&sm.k[0][0][0]) + (warp - 4) * 192;
+          float* sc_nu = sc_mu + 128;
+          const float4 m4 = reinterpret_cast<const float4*>(p.tail_mu + abase * 128)[lane];
+          const float4 q4 = reinterpret_cast<const float4*>(p.qanchor + abase * 128)[lane];
+          float qm = fmaf(m4.x, q4.x, fmaf(m4.y, q4.y, fmaf(m4.z, q4.z, m4.w * q4.w)));
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-              const int dd = 8 * c8 + 2 * e;
-              delta = fmaf(f.x - qa[dd], mu[dd], delta);
-              delta = fmaf(f.y - qa[dd + 1], mu[dd + 1], delta);
+          for (int o = 16; o > 0; o >>= 1) qm += __shfl_xor_sync(0xffffffffu, qm, o);
+          reinterpret_cast<float4*>(sc_mu)[lane] = m4;
+          if (lane < 16)
+            reinterpret_cast<float4*>(sc_nu)[lane] = reinterpret_cast<const float4*>(p.tail_nu + abase * 128 + 64 * wg)[lane];
+          __syncwarp();
+          if (row_valid) {
+            float dot = 0.f;
+            const uint32_t q_row = smem_u32(&sm.q[0][0]) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll 4
+            for (int c8 = 0; c8 < 16; ++c8) {
+              const uint32_t addr = q_row + (c8 >> 3) * kTileBytes + ((((uint32_t)c8 & 7u) ^ ((uint32_t)r & 7u)) << 4);
+              uint32_t w4[4];
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
+                           : "r"(addr));
+              const float4 ma = reinterpret_cast<const float4*>(sc_mu)[2 * c8];
+              const float4 mb = reinterpret_cast<const float4*>(sc_mu)[2 * c8 + 1];
+              const float mu8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                dot = fmaf(f.x, mu8[2 * e], dot);
+                dot = fmaf(f.y, mu8[2 * e + 1], dot);
+              }
             }
+            const float lz2 = (logz + kScale * (dot - qm)) * kLog2e;  // log2 of Zhat_i
+            const float M = fmaxf(m_ref, lz2);
+            const float eo = ex2(m_ref - M);
+            tail_w = ex2(lz2 - M);
+            const float den = l_tot * eo + tail_w;
+            scale_o = eo / den;
+            tail_w = tail_w / den;
+            nu = sc_nu;
           }
-          const float lz2 = (logz + kScale * delta) * kLog2e;  // log2 of Zhat_i
-          const float M = fmaxf(m_ref, lz2);
-          const float eo = ex2(m_ref - M);
-          tail_w = ex2(lz2 - M);
-          const float den = l_tot * eo + tail_w;
-          scale_o = eo / den;
-          tail_w = tail_w / den;
-          nu = p.tail_nu + abase * 128 + 64 * wg;
         }
       }
       // O_self columns 64 wg.. and O_other columns 64 wg.. (the other accumulator's same columns)
@@ -706,6 +725,14 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  if (p.unit_times && tid == 0) {
+    unsigned smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    unsigned long long* u = p.unit_times + 3 * (size_t)blockIdx.x;
+    u[0] = sm.t_start;
+    u[1] = globaltimer();
+    u[2] = smid;
   }
 }
 

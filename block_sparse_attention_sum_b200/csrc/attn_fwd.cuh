@@ -21,6 +21,8 @@ struct FwdParams {
   float* part_ml;
   size_t part_rows_bh;       // BH * QT * 128: rows of one split's partial state
   int* status;               // device status word
+  // optional per-CTA timing (nullptr: off): [3 CTA]: start and end of %globaltimer (ns), SM id
+  unsigned long long* unit_times;
   // Sol-Attn2 tail (unused by Sol-Attn)
   const float* qanchor;      // [BH][Na][128]
   const float* tail_logz;    // [BH][Na]

@@ -30,6 +30,8 @@ EXPORTS = [
     "sol_attn_set_kernel_timing",
     "sol_attn_last_kernel_ms",
     "sol_attn_kernel_ms_sum",
+    "sol_attn_set_unit_timing",
+    "sol_attn_last_unit_times",
     "sol_attn_last_launch_count",
     "sol_attn_release_workspace",
     "sol_attn_fwd_noalloc",
@@ -132,6 +134,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_last_kernel_ms.restype = f
     lib.sol_attn_kernel_ms_sum.argtypes = [i]
     lib.sol_attn_kernel_ms_sum.restype = f
+    lib.sol_attn_set_unit_timing.argtypes = [i]
+    lib.sol_attn_set_unit_timing.restype = i
+    lib.sol_attn_last_unit_times.argtypes = [vp, i, ctypes.POINTER(ctypes.c_int)]
+    lib.sol_attn_last_unit_times.restype = i
     lib.sol_attn_last_launch_count.argtypes = []
     lib.sol_attn_last_launch_count.restype = i
     lib.sol_attn_release_workspace.argtypes = []
@@ -326,6 +332,23 @@ def debug_route(q, k, tau=1.0, sink_start=-1, sink_tokens=0, stream=None, thresh
                                          _stream_handle(stream))
     _check(rc)
     return mask, thresh
+
+
+def set_unit_timing(enable: bool) -> None:
+    _check(load_library().sol_attn_set_unit_timing(1 if enable else 0))
+
+
+def last_unit_times():
+    """Per-CTA (start ns, end ns, SM id) of the last timed fused launch, as an int64 array [units, 3]."""
+    import numpy as np
+
+    lib = load_library()
+    n = ctypes.c_int()
+    probe = np.zeros(3, dtype=np.uint64)
+    _check(lib.sol_attn_last_unit_times(probe.ctypes.data, 0, ctypes.byref(n)))
+    buf = np.zeros(3 * n.value, dtype=np.uint64)
+    _check(lib.sol_attn_last_unit_times(buf.ctypes.data, n.value, ctypes.byref(n)))
+    return buf.reshape(n.value, 3).astype(np.int64)
 
 
 def last_stats():

@@ -189,6 +189,21 @@ int sol_attn_set_kernel_timing(int enable);
 float sol_attn_last_kernel_ms(void);
 float sol_attn_kernel_ms_sum(int n);
 
+/*
+ * Per-CTA timing of the fused attention kernel (measurement only; the pages have no counterpart).
+ * With sol_attn_set_unit_timing(1), every later BF16 forward call records, for each CTA (work unit:
+ * one 128-row query tile, or one split-KV share of it) of its fused launch, the %globaltimer value
+ * at its start and at its end (nanoseconds) and the SM it ran on.  sol_attn_last_unit_times
+ * synchronises the last call's stream and copies min(max_units, CTAs) records of three unsigned
+ * 64-bit values (start, end, SM id), in CTA order, to the HOST array `host`; *units receives the
+ * CTA count.  The first enabled call allocates a device buffer (library-owned, kept until the
+ * process exits).  Off by default; costs two stores per CTA when on.  The FP8 entry points do not
+ * record.  Errors: SOL_ERR_NULL for NULL pointers, SOL_ERR_LAUNCH when no timed
+ * launch ran.
+ */
+int sol_attn_set_unit_timing(int enable);
+int sol_attn_last_unit_times(unsigned long long* host, int max_units, int* units);
+
 /* Number of kernels the most recent forward call launched. */
 int sol_attn_last_launch_count(void);
 

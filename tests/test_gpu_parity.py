@@ -159,6 +159,26 @@ def test_stream_and_stats_and_timing():
     assert sa.last_launch_count() == 7
 
 
+def test_unit_timing_records_every_work_unit():
+    """Per-CTA timing of the fused kernel: one record per 128-row query tile, each inside the launch
+    window, on a valid SM, and the output unchanged by the recording."""
+    q, k, v = _to_gpu(*iid_qkv(2, 3000, 3, seed=8))
+    ref = sa.sol_attn_fwd(q, k, v, 1.0)
+    sa.set_unit_timing(True)
+    try:
+        out = sa.sol_attn_fwd(q, k, v, 1.0)
+        torch.cuda.synchronize()
+        ut = sa.last_unit_times()
+    finally:
+        sa.set_unit_timing(False)
+    assert torch.equal(out, ref)
+    Nb = (3000 + 63) // 64
+    assert ut.shape == (2 * 3 * ((Nb + 1) // 2), 3)
+    assert (ut[:, 1] > ut[:, 0]).all() and (ut[:, 0] > 0).all()
+    assert (ut[:, 1].max() - ut[:, 0].min()) < 1e9                  # one launch, well under a second
+    assert ((ut[:, 2] >= 0) & (ut[:, 2] < torch.cuda.get_device_properties(0).multi_processor_count)).all()
+
+
 @pytest.mark.parametrize("name", ["tiny", "wan"])
 def test_diagonal_threshold_estimator(name):
     """thresh_type="diag" (appendix "Diagonal threshold estimator") against the oracle."""
