@@ -55,6 +55,18 @@ struct DeviceState {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
+
+// Host-buffer pipeline of one device: three streams (copies in, compute, copies out), two sets of
+// device staging buffers for (b, head-chunk) slices, and the events that order them.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+  cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+  char* buf[2] = {};
+  size_t buf_bytes = 0;   // bytes of one set (q, k, v, out slices)
+};
+std::mutex g_host_mu;     // one host-buffer call at a time (they share the staging buffers)
+HostPipe g_pipe[kMaxDevices];
 bool g_timing = false;
 bool g_unit_timing = false;
 int g_last_device = -1;
@@ -316,12 +328,18 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   return check_launch("routing kernels");
 }
 
-// Validates the options against the sequence length; sets *diag, *splits and *fp8.
-int check_options(const sol_attn_options* o, int N, bool* diag, int* splits, bool* fp8) {
+// Validates the options against the sequence length; sets *diag, *splits, *fp8 and *one_block.
+int check_options(const sol_attn_options* o, int N, bool* diag, int* splits, bool* fp8, bool* one_block = nullptr) {
   *diag = false;
   *splits = 1;
   *fp8 = false;
+  if (one_block) *one_block = false;
   if (!o) return SOL_OK;
+  if (o->m_tile != 0 && o->m_tile != 64 && o->m_tile != 128)
+    return fail(SOL_ERR_OPTION, "m_tile must be 0, 64 or 128 (got %d)", o->m_tile);
+  if (o->m_tile == 64 && o->precision == SOL_PRECISION_FP8)
+    return fail(SOL_ERR_OPTION, "m_tile 64 is available on the BF16 path only");
+  if (one_block) *one_block = o->m_tile == 64;
   if (o->precision != SOL_PRECISION_BF16 && o->precision != SOL_PRECISION_FP8)
     return fail(SOL_ERR_OPTION, "unknown precision %d", o->precision);
   *fp8 = o->precision == SOL_PRECISION_FP8;
@@ -349,10 +367,11 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
             int sink_tokens, const sol_attn_options* opts, void* stream, bool sol2, bool fp8 = false) {
   int rc = validate(q, k, v, out, true, B, N, H, tau, sink_start, sink_tokens);
   if (rc) return rc;
-  bool diag, opt_fp8;
+  bool diag, opt_fp8, one_block;
   int splits;
-  if ((rc = check_options(opts, N, &diag, &splits, &opt_fp8))) return rc;
+  if ((rc = check_options(opts, N, &diag, &splits, &opt_fp8, &one_block))) return rc;
   fp8 = fp8 || opt_fp8;
+  if (fp8 && one_block) return fail(SOL_ERR_OPTION, "m_tile 64 is available on the BF16 path only");
   if (sol2 && splits > 1) return fail(SOL_ERR_OPTION, "kv_splits > 1 is available for Sol-Attn only");
   if (fp8 && splits > 1) return fail(SOL_ERR_OPTION, "kv_splits > 1 is not available on the FP8 path");
   std::lock_guard<std::mutex> lock(g_mu);
@@ -419,7 +438,8 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   p.QT = s.QT;
   p.mask = w.mask;
   p.qt_begin = 0;
-  p.qt_count = s.QT;
+  p.unit_blocks = one_block ? 1 : 2;
+  p.qt_count = one_block ? s.Nb : s.QT;   // work units per (b, h)
   p.row_lo = 0;
   p.row_hi = N;
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -432,8 +452,9 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   p.part_o = part_o;
   p.part_ml = part_ml;
   p.part_rows_bh = rows_bh;
+  const int grid = s.BH * p.qt_count * splits;
   if (g_unit_timing && !fp8) {
-    const size_t units = (size_t)s.BH * s.QT * splits;
+    const size_t units = (size_t)grid;
     if (d->unit_cap < units) {
       if (d->unit_buf) {
         cudaDeviceSynchronize();
@@ -461,7 +482,7 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
     const Fp8Params fp{f8.sq, f8.sk, f8.skbar, f8.sv, fp8_rows_padded(s) / 64};
     e = launch_attn_fwd_fp8(maps, p, fp, s.BH * s.QT, sol2, st);
   } else {
-    e = launch_attn_fwd(maps, p, s.BH * s.QT * splits, sol2, st);
+    e = launch_attn_fwd(maps, p, grid, sol2, st);
   }
   if (e != cudaSuccess) return fail(SOL_ERR_LAUNCH, "fused attention launch: %s", cudaGetErrorString(e));
   if (splits > 1) {
@@ -558,6 +579,102 @@ __global__ void wait_timeout_selftest_kernel(int* status) {
 
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 
+}  // namespace sol
+
+namespace sol {
+namespace {
+
+// The host-buffer entry points: heads are independent problems, so the (b, head-chunk) slices are
+// pipelined: the strided copy of slice c + 1 into the device overlaps the attention of slice c and
+// the copy of slice c - 1 back to the host.
+int host_pipeline(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                  int sink_start, int sink_tokens, const sol_attn_options* opts, int heads_per_chunk, bool sol2) {
+  if (!q || !k || !v || !out) return fail(SOL_ERR_NULL, "q, k, v and out must be non-NULL");
+  if (B <= 0 || N <= 0 || H <= 0) return fail(SOL_ERR_SHAPE, "B, N, H must be positive (got %d, %d, %d)", B, N, H);
+  if ((long long)B * N * H * kHeadDim > (1ll << 40)) return fail(SOL_ERR_SHAPE, "sizes out of the supported range");
+  if (heads_per_chunk < 0) return fail(SOL_ERR_SHAPE, "heads_per_chunk must be >= 0");
+  const int hc = heads_per_chunk > 0 ? std::min(heads_per_chunk, H) : std::max(1, (H + 7) / 8);
+  const size_t row = (size_t)H * kHeadDim * 2;            // bytes per token of the host tensors
+  const size_t crow = (size_t)hc * kHeadDim * 2;          // bytes per token of one slice
+  const size_t slice = (size_t)N * crow;
+  std::lock_guard<std::mutex> hlock(g_host_mu);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return fail(SOL_ERR_DEVICE, "no current CUDA device");
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    bool okc = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; i < 2 && okc; ++i)
+      okc = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!okc) {
+      cudaGetLastError();
+      return fail(SOL_ERR_DEVICE, "stream / event creation failed");
+    }
+    hp.ready = true;
+  }
+  const size_t need = 4 * align_up(slice, 256);
+  if (hp.buf_bytes < need) {
+    for (int i = 0; i < 2; ++i) {
+      if (hp.buf[i]) {
+        cudaStreamSynchronize(hp.out);
+        cudaFree(hp.buf[i]);
+      }
+      hp.buf[i] = nullptr;
+    }
+    hp.buf_bytes = 0;
+    for (int i = 0; i < 2; ++i)
+      if (cudaMalloc(&hp.buf[i], need) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(SOL_ERR_ALLOC, "staging buffers of %zu bytes failed", 2 * need);
+      }
+    hp.buf_bytes = need;
+  }
+  const int chunks_per_b = (H + hc - 1) / hc;
+  const int nchunks = B * chunks_per_b;
+  int rc = SOL_OK;
+  for (int c = 0; c < nchunks && rc == SOL_OK; ++c) {
+    const int i = c & 1;
+    const int b = c / chunks_per_b, h0 = (c % chunks_per_b) * hc, hn = std::min(hc, H - h0);
+    const size_t cw = (size_t)hn * kHeadDim * 2;          // bytes per token of this slice
+    char* base = hp.buf[i];
+    char* dq = base;
+    char* dk = base + align_up(slice, 256);
+    char* dv = base + 2 * align_up(slice, 256);
+    char* dout = base + 3 * align_up(slice, 256);
+    const size_t hoff = ((size_t)b * N * H + h0) * kHeadDim * 2;
+    // slice c reuses the buffers of slice c - 2: its compute read them and its output left them
+    if (c >= 2 && (cudaStreamWaitEvent(hp.in, hp.comp_done[i], 0) != cudaSuccess ||
+                   cudaStreamWaitEvent(hp.in, hp.out_done[i], 0) != cudaSuccess)) {
+      rc = fail(SOL_ERR_LAUNCH, "stream ordering failed");
+      break;
+    }
+    if (cudaMemcpy2DAsync(dq, cw, static_cast<const char*>(q) + hoff, row, cw, N, cudaMemcpyHostToDevice, hp.in) != cudaSuccess ||
+        cudaMemcpy2DAsync(dk, cw, static_cast<const char*>(k) + hoff, row, cw, N, cudaMemcpyHostToDevice, hp.in) != cudaSuccess ||
+        cudaMemcpy2DAsync(dv, cw, static_cast<const char*>(v) + hoff, row, cw, N, cudaMemcpyHostToDevice, hp.in) != cudaSuccess ||
+        cudaEventRecord(hp.in_done[i], hp.in) != cudaSuccess || cudaStreamWaitEvent(hp.comp, hp.in_done[i], 0) != cudaSuccess) {
+      rc = fail(SOL_ERR_LAUNCH, "host-to-device copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+      break;
+    }
+    rc = forward(dq, dk, dv, dout, 1, N, hn, tau, sink_start, sink_tokens, opts, hp.comp, sol2);
+    if (rc) break;
+    if (cudaEventRecord(hp.comp_done[i], hp.comp) != cudaSuccess || cudaStreamWaitEvent(hp.out, hp.comp_done[i], 0) != cudaSuccess ||
+        cudaMemcpy2DAsync(static_cast<char*>(out) + hoff, row, dout, cw, cw, N, cudaMemcpyDeviceToHost, hp.out) != cudaSuccess ||
+        cudaEventRecord(hp.out_done[i], hp.out) != cudaSuccess) {
+      rc = fail(SOL_ERR_LAUNCH, "device-to-host copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+      break;
+    }
+  }
+  // the call returns with the output in host memory (or after an error, with nothing in flight)
+  const bool synced = cudaStreamSynchronize(hp.in) == cudaSuccess && cudaStreamSynchronize(hp.comp) == cudaSuccess &&
+                      cudaStreamSynchronize(hp.out) == cudaSuccess;
+  if (rc == SOL_OK && !synced) rc = fail(SOL_ERR_LAUNCH, "synchronisation failed: %s", cudaGetErrorString(cudaGetLastError()));
+  return rc;
+}
+
+}  // namespace
 }  // namespace sol
 
 using namespace sol;
@@ -734,17 +851,24 @@ int sol_attn_last_launch_count(void) {
 }
 
 void sol_attn_release_workspace(void) {
+  std::lock_guard<std::mutex> hlock(g_host_mu);
   std::lock_guard<std::mutex> lock(g_mu);
   int cur = -1;
   cudaGetDevice(&cur);
   for (int i = 0; i < kMaxDevices; ++i) {
     DeviceState& d = g_dev[i];
-    if (!d.ws) continue;
+    HostPipe& hp = g_pipe[i];
+    if (!d.ws && !hp.buf[0]) continue;
     cudaSetDevice(i);
     cudaDeviceSynchronize();
-    cudaFree(d.ws);
+    if (d.ws) cudaFree(d.ws);
     d.ws = nullptr;
     d.ws_bytes = 0;
+    for (int j = 0; j < 2; ++j) {
+      if (hp.buf[j]) cudaFree(hp.buf[j]);
+      hp.buf[j] = nullptr;
+    }
+    hp.buf_bytes = 0;
   }
   if (cur >= 0) cudaSetDevice(cur);
 }
@@ -794,6 +918,18 @@ int sol_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, 
     if (rc) return rc;
   }
   return SOL_OK;
+}
+
+int sol_attn_fwd_host(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                      int sink_start, int sink_tokens, const sol_attn_options* opts, int heads_per_chunk) {
+  g_err[0] = 0;
+  return host_pipeline(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, opts, heads_per_chunk, false);
+}
+
+int sol_attn2_fwd_host(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                       int sink_start, int sink_tokens, const sol_attn_options* opts, int heads_per_chunk) {
+  g_err[0] = 0;
+  return host_pipeline(q, k, v, out, B, N, H, tau, sink_start, sink_tokens, opts, heads_per_chunk, true);
 }
 
 int sol_attn_fwd_fp8(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,

@@ -144,8 +144,9 @@ __global__ void __launch_bounds__(384, 1)
   const int unit = (int)blockIdx.x / p.kv_splits, split = (int)blockIdx.x % p.kv_splits;
   const int bh = unit / p.qt_count, qt = p.qt_begin + unit % p.qt_count;
   const int b = bh / p.H, h = bh % p.H;
-  const int qb0 = 2 * qt;
-  const bool has_hi = qb0 + 1 < p.Nb;
+  const bool one_block = p.unit_blocks == 1;   // m_tile 64: one query block, rows 64..127 idle
+  const int qb0 = one_block ? qt : 2 * qt;
+  const bool has_hi = !one_block && qb0 + 1 < p.Nb;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -450,7 +451,7 @@ __global__ void __launch_bounds__(384, 1)
     const int hf = r >> 6;
     const int qi = qb0 + hf;
     const int tok = 64 * qb0 + r;
-    const bool row_valid = tok >= p.row_lo && tok < p.row_hi;
+    const bool row_valid = (r < 64 || has_hi) && tok >= p.row_lo && tok < p.row_hi;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t o_addr = lane_addr + kColO + 128 * wg;
     const uint32_t* mrow = p.mask + ((size_t)bh * p.Nb + min(qi, p.Nb - 1)) * p.Nw;

@@ -10,7 +10,9 @@ namespace sol {
 struct FwdParams {
   int N, H, Nb, Nw, Na, QT;
   const uint32_t* mask;      // [BH][Nb][Nw]
-  int qt_begin, qt_count;    // query tiles (pairs of query blocks) qt_begin .. + qt_count - 1 of each (b, h)
+  int qt_begin, qt_count;    // work units qt_begin .. + qt_count - 1 of each (b, h)
+  int unit_blocks;           // query blocks per work unit: 1 (unit u = block u) or 2 (0 also means 2:
+                             // unit u = blocks 2u, 2u + 1)
   int row_lo, row_hi;        // token rows [row_lo, row_hi) are written; the others are computed only
   __nv_bfloat16* out;        // [B][N][H][128]
   // split-KV (kv_splits > 1): CTA s of a query tile takes the s-th contiguous share of its key

@@ -40,6 +40,8 @@ EXPORTS = [
     "sol_attn_dense_rows",
     "sol_attn_set_workspace_limit",
     "sol_attn_selftest_wait_timeout",
+    "sol_attn_fwd_host",
+    "sol_attn2_fwd_host",
     "sol_attn_fwd_fp8",
     "sol_attn2_fwd_fp8",
     "sol_attn_expcast_host",
@@ -62,12 +64,14 @@ class Options(ctypes.Structure):
 
     _fields_ = [("thresh_type", ctypes.c_int), ("n_extra_sinks", ctypes.c_int),
                 ("extra_sink_start", ctypes.c_int * MAX_EXTRA_SINKS), ("extra_sink_tokens", ctypes.c_int * MAX_EXTRA_SINKS),
-                ("kv_splits", ctypes.c_int), ("precision", ctypes.c_int), ("reserved", ctypes.c_int * 4)]
+                ("kv_splits", ctypes.c_int), ("precision", ctypes.c_int), ("m_tile", ctypes.c_int),
+                ("reserved", ctypes.c_int * 3)]
 
 
-def _options(thresh_type: str, extra_sinks=(), kv_splits: int = 1, precision: str = "bf16"):
+def _options(thresh_type: str, extra_sinks=(), kv_splits: int = 1, precision: str = "bf16", m_tile: int = 128):
     """extra_sinks: up to MAX_EXTRA_SINKS (start, tokens) token ranges made exact for every query;
-    kv_splits: split-KV shares per query tile (1 = off); precision: "bf16" or "fp8" (E4M3 + ExpCast)."""
+    kv_splits: split-KV shares per query tile (1 = off); precision: "bf16" or "fp8" (E4M3 + ExpCast);
+    m_tile: query rows per work unit of the fused kernel (128: two query blocks, 64: one)."""
     if thresh_type not in THRESH_TYPES:
         raise ValueError(f"thresh_type must be one of {sorted(THRESH_TYPES)}")
     if precision not in PRECISIONS:
@@ -80,6 +84,7 @@ def _options(thresh_type: str, extra_sinks=(), kv_splits: int = 1, precision: st
     o.n_extra_sinks = len(extra_sinks)
     o.kv_splits = int(kv_splits)
     o.precision = PRECISIONS[precision]
+    o.m_tile = int(m_tile)
     for e, (start, tokens) in enumerate(extra_sinks):
         o.extra_sink_start[e] = int(start)
         o.extra_sink_tokens[e] = int(tokens)
@@ -154,6 +159,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn_set_workspace_limit.restype = None
     lib.sol_attn_selftest_wait_timeout.argtypes = [vp]
     lib.sol_attn_selftest_wait_timeout.restype = i
+    host_args = [vp, vp, vp, vp, i, i, i, f, i, i, op, i]
+    lib.sol_attn_fwd_host.argtypes = host_args
+    lib.sol_attn_fwd_host.restype = i
+    lib.sol_attn2_fwd_host.argtypes = host_args
+    lib.sol_attn2_fwd_host.restype = i
     lib.sol_attn_fwd_fp8.argtypes = ex_args
     lib.sol_attn_fwd_fp8.restype = i
     lib.sol_attn2_fwd_fp8.argtypes = ex_args
@@ -176,11 +186,11 @@ def _stream_handle(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _check_qkv(q, k, v=None):
+def _check_qkv(q, k, v=None, host=False):
     ts = [q, k] if v is None else [q, k, v]
     for t in ts:
-        if not isinstance(t, torch.Tensor) or not t.is_cuda:
-            raise ValueError("q, k, v must be CUDA tensors")
+        if not isinstance(t, torch.Tensor) or t.is_cuda == host:
+            raise ValueError("q, k, v must be " + ("CPU" if host else "CUDA") + " tensors")
         if t.dtype != torch.bfloat16 or t.dim() != 4 or t.shape[-1] != HEAD_DIM or not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous BF16 [B, N, H, 128] (BTHD)")
         if t.shape != q.shape or t.device != q.device:
@@ -189,7 +199,7 @@ def _check_qkv(q, k, v=None):
 
 
 def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type="exact", extra_sinks=(),
-         kv_splits=1, precision="bf16"):
+         kv_splits=1, precision="bf16", m_tile=128):
     B, N, H = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
@@ -199,8 +209,8 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
     args = [q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, float(tau), int(sink_start),
             int(sink_tokens)]
     with torch.cuda.device(q.device):
-        if thresh_type != "exact" or extra_sinks or kv_splits != 1 or precision != "bf16":
-            opts = _options(thresh_type, extra_sinks, kv_splits, precision)
+        if thresh_type != "exact" or extra_sinks or kv_splits != 1 or precision != "bf16" or m_tile != 128:
+            opts = _options(thresh_type, extra_sinks, kv_splits, precision, m_tile)
             rc = getattr(lib, fn_name + "_ex")(*args, ctypes.byref(opts), _stream_handle(stream))
         else:
             rc = getattr(lib, fn_name)(*args, _stream_handle(stream))
@@ -209,17 +219,46 @@ def _fwd(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_typ
 
 
 def sol_attn_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
-                 extra_sinks=(), kv_splits=1, precision="bf16"):
+                 extra_sinks=(), kv_splits=1, precision="bf16", m_tile=128):
     """Sol-Attn forward through the C ABI; returns ``out`` (BF16 [B, N, H, 128])."""
     return _fwd("sol_attn_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks,
-                kv_splits, precision)
+                kv_splits, precision, m_tile)
 
 
 def sol_attn2_fwd(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None, thresh_type="exact",
-                  extra_sinks=(), precision="bf16"):
+                  extra_sinks=(), precision="bf16", m_tile=128):
     """Sol-Attn2 complementary-tail forward through the C ABI; returns ``out``."""
     return _fwd("sol_attn2_fwd", q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks,
-                precision=precision)
+                precision=precision, m_tile=m_tile)
+
+
+def _fwd_host(fn_name, q, k, v, tau, sink_start, sink_tokens, out, thresh_type, extra_sinks, heads_per_chunk):
+    B, N, H = _check_qkv(q, k, v, host=True)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device.type != "cpu":
+        raise ValueError("out must be a contiguous BF16 CPU tensor shaped like q")
+    opts = _options(thresh_type, extra_sinks)
+    lib = load_library()
+    rc = getattr(lib, fn_name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, float(tau),
+                               int(sink_start), int(sink_tokens), ctypes.byref(opts), int(heads_per_chunk))
+    _check(rc)
+    return out
+
+
+def sol_attn_fwd_host(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, thresh_type="exact", extra_sinks=(),
+                      heads_per_chunk=0):
+    """Sol-Attn forward of HOST (CPU) tensors, copies pipelined with the computation on the current
+    CUDA device; pin the tensors for overlap.  Returns ``out`` (a CPU tensor)."""
+    return _fwd_host("sol_attn_fwd_host", q, k, v, tau, sink_start, sink_tokens, out, thresh_type, extra_sinks,
+                     heads_per_chunk)
+
+
+def sol_attn2_fwd_host(q, k, v, tau=1.0, sink_start=-1, sink_tokens=0, out=None, thresh_type="exact", extra_sinks=(),
+                       heads_per_chunk=0):
+    """Sol-Attn2 forward of HOST (CPU) tensors (see sol_attn_fwd_host)."""
+    return _fwd_host("sol_attn2_fwd_host", q, k, v, tau, sink_start, sink_tokens, out, thresh_type, extra_sinks,
+                     heads_per_chunk)
 
 
 def _fwd_fp8(fn_name, q, k, v, tau, sink_start, sink_tokens, out, stream, thresh_type, extra_sinks):

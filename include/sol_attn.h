@@ -95,6 +95,16 @@ typedef enum {
  *                      sol_attn_fwd_varlen run the FP8 path of sol_attn_fwd_fp8 / sol_attn2_fwd_fp8;
  *                      it cannot be combined with kv_splits > 1.  The routing (and so
  *                      sol_attn_debug_route_ex) is the same for both.
+ *   m_tile             query rows per work unit of the fused kernel: 0 or 128 (default), two
+ *                      adjacent 64-token query blocks per unit, which walk the union of their exact
+ *                      sets (a key block exact for only one of them is computed for both rows and
+ *                      masked for the other: the union-tile waste); 64, one query block per unit,
+ *                      which walks only its own exact set (no union waste) at the same tensor cost
+ *                      per tile as two blocks, so it pays only where the union waste exceeds one
+ *                      half (the tensor-core tile stays M = 128; its second half is idle).  The
+ *                      Sol-Attn README's per-shape tuning knobs ("Long-sequence tuning on H100")
+ *                      motivate it.  Results equal the default up to FP32 rounding.  BF16 path
+ *                      only: an FP8 precision with m_tile 64 returns SOL_ERR_OPTION.
  */
 typedef struct {
   int thresh_type;
@@ -103,7 +113,8 @@ typedef struct {
   int extra_sink_tokens[SOL_MAX_EXTRA_SINKS];
   int kv_splits;
   int precision;
-  int reserved[4];
+  int m_tile;
+  int reserved[3];
 } sol_attn_options;
 
 /*
@@ -294,6 +305,29 @@ void sol_attn_set_workspace_limit(size_t bytes);
  * device.
  */
 int sol_attn_selftest_wait_timeout(void* stream);
+
+/*
+ * Host-buffer entry points (the Sol-Attn README's sol_attn call takes and returns tensors; these
+ * take them in host memory).  q, k, v and out are HOST pointers to [B, N, H, 128] BF16 arrays (BTHD,
+ * contiguous; no alignment needed); the computation is sol_attn_fwd_ex / sol_attn2_fwd_ex (`opts`
+ * may be NULL) and the call blocks until `out` holds the result.
+ *   - Heads are independent problems, so the call splits the work into (b, head-chunk) slices of
+ *     heads_per_chunk heads (0: ceil(H / 8)) and pipelines them on three internal streams of the
+ *     current device: the strided copy of slice c + 1 into device memory, the attention of slice c
+ *     and the copy of slice c - 1 back to the host overlap.  Overlap needs page-locked host memory
+ *     (cudaHostAlloc / cudaHostRegister); pageable buffers give the same result without it.
+ *   - Each slice is a separate call (its own routing, launches and statistics): the result equals
+ *     sol_attn_fwd_ex on device copies of the tensors bit for bit.
+ *   - The library keeps two sets of device staging buffers (4 x N x heads_per_chunk x 256 bytes
+ *     each) besides its workspace, until sol_attn_release_workspace.  Calls are serialised.
+ *   - Errors: SOL_ERR_NULL / SOL_ERR_SHAPE for bad arguments, SOL_ERR_ALLOC when staging buffers
+ *     cannot be allocated, SOL_ERR_LAUNCH when a copy fails, otherwise the first failing slice's
+ *     status (nothing is left in flight).
+ */
+int sol_attn_fwd_host(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                      int sink_start, int sink_tokens, const sol_attn_options* opts, int heads_per_chunk);
+int sol_attn2_fwd_host(const void* q, const void* k, const void* v, void* out, int B, int N, int H, float tau,
+                       int sink_start, int sink_tokens, const sol_attn_options* opts, int heads_per_chunk);
 
 /*
  * FP8 (E4M3) + ExpCast forward ("Sol-Attn2" draft, section "FP8 quantization and ExpCast").  Same

@@ -65,8 +65,15 @@ def test_invalid_options_are_rejected_on_the_host(lib):
     rc = lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None)
     assert rc == -10
     opts = sa.Options(1)
-    opts.reserved[3] = 1
+    opts.reserved[2] = 1
     assert lib.sol_attn2_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa._options("exact", m_tile=96)           # m_tile is 0, 64 or 128
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    assert b"m_tile" in lib.sol_attn_last_error()
+    opts = sa._options("exact", precision="fp8", m_tile=64)   # one-block units: BF16 path only
+    assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
+    opts = sa._options("exact", m_tile=64)
+    assert lib.sol_attn_fwd_fp8(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
     opts = sa._options("exact", [(10, 0)])          # an extra sink needs tokens > 0
     assert lib.sol_attn_fwd_ex(16, 16, 16, 1 << 40, 1, 128, 2, 1.0, -1, 0, ctypes.byref(opts), None) == -10
     opts = sa._options("exact", [(128, 4)])         # start must be < N
@@ -98,7 +105,8 @@ def test_options_struct_matches_the_header():
     assert "#define SOL_MAX_KV_SPLITS 8" in text and sa.MAX_KV_SPLITS == 8
     assert ctypes.sizeof(sa.Options) == 16 * 4
     assert "SOL_PRECISION_BF16 = 0" in text and "SOL_PRECISION_FP8 = 1" in text and sa.PRECISIONS == {"bf16": 0, "fp8": 1}
-    assert sa.Options.precision.offset == 11 * 4 and sa.Options.reserved.offset == 12 * 4
+    assert sa.Options.precision.offset == 11 * 4 and sa.Options.m_tile.offset == 12 * 4
+    assert sa.Options.reserved.offset == 13 * 4 and "int m_tile;\n  int reserved[3];" in text
 
 
 def test_dense_rows_host_validation(lib):

@@ -271,6 +271,49 @@ def test_split_kv(case, kv_splits):
     assert (out.float() - one.float()).abs().max().item() <= 1.6e-2
 
 
+@pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
+@pytest.mark.parametrize("case", [("n129", 1, 129, 2, 1.0, -1, 0), ("n1000_b2", 2, 1000, 2, 1.0, -1, 0),
+                                  ("n1000_interior_sink", 1, 1000, 2, 1.5, 300, 200),
+                                  ("n4000_high_tau", 1, 4000, 2, 3.0, -1, 0)], ids=lambda c: c[0])
+def test_m_tile_64(case, entry):
+    """m_tile = 64 (one query block per work unit, README per-shape tuning): the oracle's result,
+    and the default tiling's up to FP32 rounding; odd and even block counts, a ragged last block."""
+    name, B, N, H, tau, ss, st = case
+    q, k, v = _small_inputs(name, B, N, H)
+    fn = getattr(orc, entry)
+    ref = fn(q, k, v, tau, ss, st)
+    qd, kd, vd = _to_gpu(q, k, v)
+    gfn = sa.sol_attn_fwd if entry == "sol_attn" else sa.sol_attn2_fwd
+    out = gfn(qd, kd, vd, tau, ss, st, m_tile=64)
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    gmask, _ = sa.debug_route(qd, kd, tau, ss, st)
+    gm = gmask.cpu().numpy()
+    skip = check_mask(gm, ref, orc.sink_block_flags(N, ss, st))
+    compare_outputs(out.float().cpu().numpy(), with_gpu_mask(fn, (q, k, v, tau, ss, st), gm, skip, ref["out"]), N)
+    default = gfn(qd, kd, vd, tau, ss, st)
+    torch.cuda.synchronize()
+    assert (out.float() - default.float()).abs().max().item() <= 1.6e-2
+
+
+@pytest.mark.parametrize("entry", ["sol_attn", "sol_attn2"])
+def test_host_buffer_entry_points_match_the_device_call(entry):
+    """sol_attn_fwd_host / sol_attn2_fwd_host: pinned host tensors in and out, (b, head-chunk) slices
+    pipelined; each slice is an independent call, so the result equals the device call bit for bit
+    (B = 2, H = 5 heads in chunks of 2, the last one short)."""
+    q, k, v = iid_qkv(2, 1500, 5, seed=19)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    host_fn = sa.sol_attn_fwd_host if entry == "sol_attn" else sa.sol_attn2_fwd_host
+    dev_fn = sa.sol_attn_fwd if entry == "sol_attn" else sa.sol_attn2_fwd
+    out = host_fn(qh, kh, vh, 1.0, 0, 64, heads_per_chunk=2)
+    ref = dev_fn(*_to_gpu(q, k, v), 1.0, 0, 64)
+    torch.cuda.synchronize()
+    assert sa.get_device_status() == 0
+    assert out.device.type == "cpu" and torch.equal(out, ref.cpu())
+    again = host_fn(q, k, v, 1.0, 0, 64)          # pageable buffers, default chunking
+    assert torch.equal(again, out)
+
+
 def test_split_kv_is_sol_attn_only():
     q, k, v = _to_gpu(*iid_qkv(1, 256, 1, seed=3))
     with pytest.raises(sa.SolAttnError):
