@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--kv-splits", type=int, default=1,
                     help="split-KV shares per 128-row query tile (Sol-Attn only; 1 = off)")
+    ap.add_argument("--m-tile", type=int, default=128, choices=[64, 128],
+                    help="query rows per work unit of the fused kernel (128: two query blocks; 64: one)")
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"],
                     help="attention products in BF16 (default) or E4M3 with ExpCast weights (sol_attn*_fwd_fp8)")
     ap.add_argument("--no-fp8-leg", action="store_true",
@@ -77,26 +79,31 @@ def max_over_ranks(values, world: int, device=None):
     return [float(x) for x in t.tolist()]
 
 
-TRAFFIC_PATH = os.path.join(ROOT, "profiles", "attn_fwd_dram_traffic.json")
-KERNEL_SOURCE = os.path.join(ROOT, "block_sparse_attention_sum_b200", "csrc", "attn_fwd.cu")
+TRAFFIC = {  # committed ncu DRAM records and the kernel source each was taken with
+    "bf16": (os.path.join(ROOT, "profiles", "attn_fwd_dram_traffic.json"),
+             os.path.join(ROOT, "block_sparse_attention_sum_b200", "csrc", "attn_fwd.cu")),
+    "fp8": (os.path.join(ROOT, "profiles", "attn_fwd_fp8_dram_traffic.json"),
+            os.path.join(ROOT, "block_sparse_attention_sum_b200", "csrc", "attn_fwd_fp8.cu")),
+}
 
 
-def kernel_source_digest() -> str:
+def kernel_source_digest(path: str) -> str:
     import hashlib
 
-    with open(KERNEL_SOURCE, "rb") as f:
+    with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()
 
 
-def measured_traffic(workload_name: str):
+def measured_traffic(workload_name: str, precision: str = "bf16"):
     """DRAM bytes per launch of the fused kernel from a committed ncu capture, if that capture was
     taken on this workload with the current kernel source (else None)."""
-    if not os.path.exists(TRAFFIC_PATH):
+    record, source = TRAFFIC[precision]
+    if not os.path.exists(record):
         return None
-    with open(TRAFFIC_PATH) as f:
+    with open(record) as f:
         rec = json.load(f)
     entry = rec.get(workload_name)
-    if not entry or entry.get("source_sha256") != kernel_source_digest():
+    if not entry or entry.get("source_sha256") != kernel_source_digest(source):
         return None
     return entry["dram_bytes_per_launch"]
 
@@ -267,7 +274,8 @@ def fp8_leg(sa, w, q, k, v, out_bf16, tau, stream, flops_step, peaks, steps):
                 "value": value, "unit": "TFLOP/s", "frac_of_peak": value / bf16_burst,
                 "frac_of_sustained_peak": value / bf16_sust,
                 "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": 2.0 * bf16_sust,
-                             "unit": "TFLOP/s", "frac": kernel_tflops / (2.0 * bf16_sust), "traffic": None,
+                             "unit": "TFLOP/s", "frac": kernel_tflops / (2.0 * bf16_sust),
+                             "traffic": measured_traffic(w.name, "fp8"),
                              "kernel": "attn_fwd_fp8_kernel", "kernel_ms": kernel_ms,
                              "peak_kind": f"e4m3 dense sustained = 2 x measured bf16 ({peaks['source']})"},
                 "gpu_launches": launches * n, "rel_l2_vs_bf16_output": rel,
@@ -448,6 +456,10 @@ def main():
     stream = torch.cuda.current_stream()
 
     extra = {"kv_splits": args.kv_splits} if args.kv_splits != 1 else {}
+    if args.m_tile != 128:
+        if fp8:
+            raise SystemExit("--m-tile 64 is available with --precision bf16 only")
+        extra["m_tile"] = args.m_tile
 
     def step():
         fn(q, k, v, tau, w.sink_start, w.sink_tokens, out=out, stream=stream, **extra)
@@ -494,18 +506,17 @@ def main():
     union_frac = union_useful_fraction(gmask.cpu().numpy())
     del gmask
 
-    # ---- end to end through the public API with host buffers (H2D inputs, D2H output each step)
+    # ---- end to end through the public API with host buffers: the host-buffer entry point, whose
+    # copies in (pinned host -> device) and out (device -> pinned host) run inside the timed region,
+    # pipelined with the computation over head slices
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not fp8 and args.kv_splits == 1 and args.m_tile == 128:
         out_h = torch.empty_like(qh).pin_memory()
         e2e_steps = max(3, min(args.steps, 10))
+        host_fn = sa.sol_attn_fwd_host if w.entry == "sol_attn" else sa.sol_attn2_fwd_host
 
         def e2e_step():
-            q.copy_(qh, non_blocking=True)
-            k.copy_(kh, non_blocking=True)
-            v.copy_(vh, non_blocking=True)
-            step()
-            out_h.copy_(out, non_blocking=True)
+            host_fn(qh, kh, vh, tau, w.sink_start, w.sink_tokens, out=out_h)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -520,7 +531,9 @@ def main():
         e2e_ms = max_over_ranks([a.elapsed_time(b) / e2e_steps], world, dev)[0]
         e2e = {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 3 * qh.numel() * qh.element_size(),
-               "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": e2e_steps}
+               "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": e2e_steps,
+               "call": host_fn.__name__ + " (pinned host tensors in and out, head slices pipelined)",
+               "matches_device_call": bool(torch.equal(out_h, out.cpu()))}
 
     peaks = load_peaks()
     # E4M3 products: the measured BF16 peak times the nominal dense FP8 / BF16 ratio (4.5 / 2.25)
@@ -530,7 +543,7 @@ def main():
     achieved = flops_step / (kernel_ms * 1e-3) / 1e12
     kname = ("attn_fwd_fp8_kernel" if fp8 else "attn_fwd_kernel") + ("<false>" if w.entry == "sol_attn" else "<true>")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sust, "unit": "TFLOP/s",
-                "frac": achieved / peak_sust, "traffic": None if fp8 else measured_traffic(w.name),
+                "frac": achieved / peak_sust, "traffic": measured_traffic(w.name, "fp8" if fp8 else "bf16"),
                 "kernel": kname + " (fused attention)",
                 "kernel_ms": kernel_ms,
                 "peak_kind": (f"e4m3 dense sustained = 2 x measured bf16 ({peaks['source']})" if fp8 else
@@ -545,6 +558,7 @@ def main():
                        "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "tau": tau,
                        "target_sparsity": w.target_sparsity, "realised_sparsity": sp,
                        "union_tile_useful_fraction": union_frac, "kv_splits": args.kv_splits,
+                       "m_tile": args.m_tile,
                        "min_row": min_row, "max_row": max_row, "scheduler": sched,
                        "precision": args.precision,
                        "parallelism": f"independent replicas x{world} (head/batch sharding, no exchange)",
@@ -557,7 +571,7 @@ def main():
 
     if world == 1 and not fp8 and not args.no_fp8_leg:
         line["fp8"] = fp8_leg(sa, w, q, k, v, out, tau, stream, flops_step, peaks, args.steps)
-    if world == 1 and not fp8 and not args.no_legs and w.name == "s64k" and args.kv_splits == 1:
+    if world == 1 and not fp8 and not args.no_legs and w.name == "s64k" and args.kv_splits == 1 and args.m_tile == 128:
         def inputs_key(x):   # workloads that differ only in tau target or sink share their inputs
             return x.input_key().split("@")[0].split("+")[0]
 
