@@ -593,7 +593,7 @@ int host_pipeline(const void* q, const void* k, const void* v, void* out, int B,
   if (B <= 0 || N <= 0 || H <= 0) return fail(SOL_ERR_SHAPE, "B, N, H must be positive (got %d, %d, %d)", B, N, H);
   if ((long long)B * N * H * kHeadDim > (1ll << 40)) return fail(SOL_ERR_SHAPE, "sizes out of the supported range");
   if (heads_per_chunk < 0) return fail(SOL_ERR_SHAPE, "heads_per_chunk must be >= 0");
-  const int hc = heads_per_chunk > 0 ? std::min(heads_per_chunk, H) : std::max(1, (H + 7) / 8);
+  const int hc = heads_per_chunk > 0 ? std::min(heads_per_chunk, H) : std::max(1, (H + 15) / 16);
   const size_t row = (size_t)H * kHeadDim * 2;            // bytes per token of the host tensors
   const size_t crow = (size_t)hc * kHeadDim * 2;          // bytes per token of one slice
   const size_t slice = (size_t)N * crow;

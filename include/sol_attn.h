@@ -312,7 +312,7 @@ int sol_attn_selftest_wait_timeout(void* stream);
  * contiguous; no alignment needed); the computation is sol_attn_fwd_ex / sol_attn2_fwd_ex (`opts`
  * may be NULL) and the call blocks until `out` holds the result.
  *   - Heads are independent problems, so the call splits the work into (b, head-chunk) slices of
- *     heads_per_chunk heads (0: ceil(H / 8)) and pipelines them on three internal streams of the
+ *     heads_per_chunk heads (0: ceil(H / 16)) and pipelines them on three internal streams of the
  *     current device: the strided copy of slice c + 1 into device memory, the attention of slice c
  *     and the copy of slice c - 1 back to the host overlap.  Overlap needs page-locked host memory
  *     (cudaHostAlloc / cudaHostRegister); pageable buffers give the same result without it.
