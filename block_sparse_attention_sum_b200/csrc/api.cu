@@ -297,7 +297,8 @@ int check_launch(const char* what) {
 // Routing prefix shared by all entry points: summaries, threshold statistics, thresholds, bitmask.
 int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                 const Shape& s, const Work& w, float tau, int sink_start, int sink_tokens, bool anchors,
-                bool diag, const sol_attn_options* opts, cudaStream_t st, int* launches) {
+                bool diag, const sol_attn_options* opts, cudaStream_t st, int* launches,
+                const Fp8Work* f8 = nullptr) {
   SinkSet sinks{};
   add_sink(s.N, sink_start, sink_tokens, &sinks);
   if (opts)
@@ -311,10 +312,13 @@ int run_routing(DeviceState& d, const __nv_bfloat16* q, const __nv_bfloat16* k, 
   if (rc) return rc;
   Work ww = w;
   ww.stats = d.stats;
+  // FP8: the summary pass also quantises Q and K and takes the heads' max |V| (cleared here)
+  if (f8 && cudaMemsetAsync(f8->vmax, 0, (size_t)s.BH * sizeof(unsigned int), st) != cudaSuccess)
+    return fail(SOL_ERR_LAUNCH, "V maximum reset failed");
   if (anchors)
-    launch_sol2_summaries(q, k, v, s, ww, st);   // Sol-Attn2: the key groups come with the key means
+    launch_sol2_summaries(q, k, v, s, ww, st, f8);   // Sol-Attn2: the key groups come with the key means
   else
-    launch_summary(q, k, v, s, ww, false, st);
+    launch_summary(q, k, v, s, ww, false, st, f8);
   launch_kstats(s, ww, st);
   launch_thresh(s, ww, tau, diag, st);
   CUtensorMap rmaps[4];
@@ -413,7 +417,9 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
   const auto* qh = static_cast<const __nv_bfloat16*>(q);
   const auto* kh = static_cast<const __nv_bfloat16*>(k);
   const auto* vh = static_cast<const __nv_bfloat16*>(v);
-  if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, diag, opts, st, &launches))) return rc;
+  if ((rc = run_routing(*d, qh, kh, vh, s, w, tau, sink_start, sink_tokens, sol2, diag, opts, st, &launches,
+                        fp8 ? &f8 : nullptr)))
+    return rc;
   if (sol2) {
     CUtensorMap tmaps[3];
     if ((rc = encode_rows(&tmaps[0], w.qanchor_h, s.Na, s)) || (rc = encode_rows(&tmaps[1], w.gk_h, 2 * s.Nb, s)) ||
@@ -425,8 +431,8 @@ int forward(const void* q, const void* k, const void* v, void* out, int B, int N
     if ((rc = check_launch("Sol-Attn2 tail kernels"))) return rc;
   }
   if (fp8) {
-    launch_quant_fp8(qh, kh, vh, s, w, f8, st);
-    launches += 3;
+    launch_quant_fp8(vh, s, w, f8, st);
+    launches += 2;
     if ((rc = check_launch("FP8 quantisation kernels"))) return rc;
   }
   FwdParams p{};

@@ -66,9 +66,13 @@ struct Work {
 // Sets the calling thread's message returned by sol_attn_last_error() (api.cu).
 void set_last_error(const char* msg);
 
-// Prep kernels (summary.cu)
+struct Fp8Work;
+
+// Prep kernels (summary.cu).  With f8, the summary pass also writes the E4M3 codes of Q and K with
+// their block scales and folds max |V| of every block into the head's maximum (f8->vmax, cleared
+// before the call).
 void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                    const Work& w, bool anchors, cudaStream_t st);
+                    const Work& w, bool anchors, cudaStream_t st, const Fp8Work* f8 = nullptr);
 void launch_kstats(const Shape& s, const Work& w, cudaStream_t st);
 void launch_thresh(const Shape& s, const Work& w, float tau, bool diag, cudaStream_t st);
 // Routing on the tensor cores (route_tc.cu); maps = qbar_hi, qbar_lo, kbar_h, kbar_lo (BF16, 3-D,
@@ -91,7 +95,7 @@ void launch_dense_mask(const Shape& s, const Work& w, int qb_lo, int qb_hi, cuda
 // Sol-Attn2 summaries (sol2_tail.cu), in place of launch_summary: query and anchor means, the mean
 // query, then key means and the two key groups of every block (three launches).
 void launch_sol2_summaries(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                           const Work& w, cudaStream_t st);
+                           const Work& w, cudaStream_t st, const Fp8Work* f8 = nullptr);
 // Sol-Attn2 tail statistics on the tensor cores (sol2_tail_tc.cu); maps = anchor means, group key
 // means, group value means (BF16, 3-D, box 64 x 128 x 1, 128-byte swizzle).
 cudaError_t launch_tail_tc(const void* maps, const Shape& s, const Work& w, int* status, cudaStream_t st);
@@ -112,7 +116,7 @@ struct Fp8Work {
 };
 // Rows of the compressed-key arrays: Nb rounded up to whole 128-row surrogate chunks.
 __host__ __device__ inline int fp8_rows_padded(const Shape& s) { return (s.Nb + 127) / 128 * 128; }
-void launch_quant_fp8(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                      const Work& w, const Fp8Work& f, cudaStream_t st);
+// V (head scale) and the compressed keys / values; Q and K come from the summary pass (f8 there).
+void launch_quant_fp8(const __nv_bfloat16* v, const Shape& s, const Work& w, const Fp8Work& f, cudaStream_t st);
 
 }  // namespace sol

@@ -7,6 +7,9 @@
 #pragma once
 #include <cstdint>
 #include <cmath>
+#ifdef __CUDACC__
+#include <cuda_bf16.h>
+#endif
 
 namespace sol {
 
@@ -124,6 +127,71 @@ __device__ __forceinline__ uint32_t to_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// X / s with s = m / 448, evaluated as (x * 448) / m: for a BF16 x the product is exact and the
+// quotient is correctly rounded, so a value that lies exactly halfway between two E4M3 numbers
+// (frequent: x and m share most of their few mantissa bits) stays exactly halfway and rounds to
+// even, as the definition asks; x / fl(m / 448) can land just off the midpoint and round the
+// other way.  m > 0.
+__device__ __forceinline__ float scaled448(float x, float m) { return (x * 448.0f) / m; }
+
+// Eight values of a block with maximum |X| = m > 0, as four E4M3 pairs in one 8-byte word.
+__device__ __forceinline__ uint2 codes8(const float (&v)[8], float m) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) w[e] = to_e4m3x2(scaled448(v[2 * e], m), scaled448(v[2 * e + 1], m));
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// The largest |x| of a 64-token block held by 256 threads (each holds four rows of 8 BF16 channels,
+// `rows`, as the block-summary kernels load them): warp shuffles, then eight warp maxima through
+// `red` (8 floats of shared memory; the call synchronises the block twice).
+__device__ __forceinline__ float block_absmax(const uint4 (&rows)[4], float* red) {
+  float m = 0.f;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&rows[r]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(p[e]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float b = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) b = fmaxf(b, red[i]);
+  __syncthreads();
+  return b;
+}
+
+// E4M3 codes of one 64-token block (one scale, s = max |X| / 448; an all-zero block keeps s = 1 and
+// zero codes) from the rows the block-summary kernels hold: this thread's rows rg + 16 r (r < 4) of
+// channels 8 c16 .. 8 c16 + 7, written to x8 ([B][N][H][128] bytes) and the scale to *scale (by
+// thread 0).  Rows past the sequence (row >= n) are not written.
+__device__ __forceinline__ void quant_block_rows(const uint4 (&rows)[4], float m, uint8_t* x8, float* scale, int N,
+                                                 int H, int b, int h, int t0, int n, int tid) {
+  const int c16 = tid & 15, rg = tid >> 4;
+  if (tid == 0) *scale = m > 0.f ? m / 448.0f : 1.0f;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int row = rg + 16 * r;
+    if (row >= n) continue;
+    float v[8];
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&rows[r]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(p[e]);
+      v[2 * e] = f.x;
+      v[2 * e + 1] = f.y;
+    }
+    *reinterpret_cast<uint2*>(x8 + (((size_t)b * N + t0 + row) * H + h) * 128 + 8 * c16) =
+        m > 0.f ? codes8(v, m) : make_uint2(0u, 0u);
+  }
 }
 #endif  // __CUDACC__
 

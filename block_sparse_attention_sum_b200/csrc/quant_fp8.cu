@@ -1,4 +1,5 @@
-// E4M3 operands of the FP8 forward.
+// E4M3 operands of the FP8 forward: V and the compressed keys / values here; Q and K are quantised
+// by the block-summary kernels in their pass over Q and K (quant_block_rows in fp8.cuh).
 //
 // Sol-Attn2 draft, section "FP8 quantization and ExpCast": one scale per 64-token block for Q and K,
 // one per head for V, s = max |X| / 448 (an all-zero block keeps s = 1), codes E4M3(X / s) rounded to
@@ -53,53 +54,6 @@ __device__ __forceinline__ void load_rows_bf16(const __nv_bfloat16* x, const Sha
     }
   }
   *amax = m;
-}
-
-// X / s with s = m / 448, evaluated as (x * 448) / m: for a BF16 x the product is exact and the
-// quotient is correctly rounded, so a value that lies exactly halfway between two E4M3 numbers
-// (frequent: x and m share most of their few mantissa bits) stays exactly halfway and rounds to
-// even, as the definition asks; x / fl(m / 448) can land just off the midpoint and round the
-// other way.  m > 0.
-__device__ __forceinline__ float scaled448(float x, float m) { return (x * 448.0f) / m; }
-
-// Eight values of a block with maximum |X| = m > 0, as four E4M3 pairs in one 8-byte word.
-__device__ __forceinline__ uint2 codes8(const float (&v)[8], float m) {
-  uint32_t w[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) w[e] = to_e4m3x2(scaled448(v[2 * e], m), scaled448(v[2 * e + 1], m));
-  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-}
-
-// grid (Nb, BH, 3): z = 0 quantises Q, z = 1 K (per 64-token block), z = 2 takes the block maximum
-// of |V| into the head's maximum (float bits of a non-negative value order like unsigned integers).
-__global__ void __launch_bounds__(256) quant_qk_kernel(const __nv_bfloat16* __restrict__ q,
-                                                       const __nv_bfloat16* __restrict__ k,
-                                                       const __nv_bfloat16* __restrict__ v, uint8_t* __restrict__ q8,
-                                                       uint8_t* __restrict__ k8, float* __restrict__ sq,
-                                                       float* __restrict__ sk, unsigned int* __restrict__ vmax,
-                                                       const Shape s) {
-  __shared__ float red[8];
-  const int j = blockIdx.x, bh = blockIdx.y, z = blockIdx.z, tid = threadIdx.x;
-  const int b = bh / s.H, h = bh % s.H, t0 = j * kBlock, n = min(kBlock, s.N - t0);
-  const __nv_bfloat16* x = z == 0 ? q : (z == 1 ? k : v);
-  float vals[4][8], amax;
-  load_rows_bf16(x, s, b, h, t0, n, tid, vals, &amax);
-  const float m = block_max_256(amax, red);
-  if (z == 2) {
-    if (tid == 0) atomicMax(vmax + bh, __float_as_uint(m));
-    return;
-  }
-  const float sc = m > 0.f ? m / 448.0f : 1.0f;
-  if (tid == 0) (z == 0 ? sq : sk)[(size_t)bh * s.Nb + j] = sc;
-  uint8_t* x8 = z == 0 ? q8 : k8;
-  const int c16 = tid & 15, rg = tid >> 4;
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int row = rg + 16 * r;
-    if (row < n)
-      *reinterpret_cast<uint2*>(x8 + (((size_t)b * s.N + t0 + row) * s.H + h) * kHeadDim + 8 * c16) =
-          m > 0.f ? codes8(vals[r], m) : make_uint2(0u, 0u);
-  }
 }
 
 // grid (Nb, BH): V with the head's scale, and the block's value mean Vbar_j (FP32 column sums over
@@ -178,11 +132,8 @@ __global__ void __launch_bounds__(256) quant_kbar_kernel(const float* __restrict
 
 }  // namespace
 
-void launch_quant_fp8(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                      const Work& w, const Fp8Work& f, cudaStream_t st) {
+void launch_quant_fp8(const __nv_bfloat16* v, const Shape& s, const Work& w, const Fp8Work& f, cudaStream_t st) {
   const int nbp = fp8_rows_padded(s);
-  cudaMemsetAsync(f.vmax, 0, (size_t)s.BH * sizeof(unsigned int), st);
-  quant_qk_kernel<<<dim3(s.Nb, s.BH, 3), 256, 0, st>>>(q, k, v, f.q8, f.k8, f.sq, f.sk, f.vmax, s);
   quant_v_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(v, f.v8, f.vbar8, f.sv, f.vmax, s, nbp);
   quant_kbar_kernel<<<dim3(nbp / 64, s.BH), 256, 0, st>>>(w.kbar, f.kbar8, f.vbar8, f.skbar, s, nbp);
 }

@@ -11,6 +11,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "fp8.cuh"
 
 namespace sol {
 
@@ -44,8 +45,11 @@ __global__ void __launch_bounds__(1024) qdir_kernel(Shape s, Work w) {
 // product) and the two 32-token anchor means of every block.  One CTA per (query block j, b, h)
 // with summary_kernel's thread mapping and summation order, so Qbar is bit-identical to the
 // Sol-Attn path's.
-__global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __restrict__ q, Shape s, Work w) {
+template <bool kQuant>
+__global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __restrict__ q, Shape s, Work w,
+                                                        Fp8Work f8) {
   __shared__ float red[8][2][kHeadDim];
+  __shared__ float qred[8];
   const int j = blockIdx.x, b = blockIdx.y / s.H, h = blockIdx.y % s.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c16 = tid & 15, rg = tid >> 4;
@@ -62,6 +66,10 @@ __global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __r
     rq[m] = r < n ? __ldg(reinterpret_cast<const uint4*>(q + ((size_t)(b * (size_t)s.N + t0 + r) * s.H + h) * kHeadDim +
                                                         8 * c16))
                   : make_uint4(0, 0, 0, 0);
+  }
+  if (kQuant) {   // the FP8 path: Q codes and the block's scale in the same pass
+    const float mq = block_absmax(rq, qred);
+    quant_block_rows(rq, mq, f8.q8, f8.sq + ((size_t)b * s.H + h) * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
   }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
@@ -124,9 +132,12 @@ __global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __r
 // decision), their sizes, key means and value means.  K and V are read once, kept in registers
 // between the block-mean reduction and the group split.  One CTA per (key block j, b, h): 16
 // threads cover a 256-byte row with 16-byte loads, 16 row groups cover the block.
+template <bool kQuant>
 __global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloat16* __restrict__ k,
-                                                                const __nv_bfloat16* __restrict__ v, Shape s, Work w) {
+                                                                const __nv_bfloat16* __restrict__ v, Shape s, Work w,
+                                                                Fp8Work f8) {
   __shared__ float red[8][4][kHeadDim];
+  __shared__ float qred[8];
   __shared__ float kbar_s[kHeadDim];
   __shared__ int n1_s;
   const int j = blockIdx.x, bh = blockIdx.y, b = bh / s.H, h = bh % s.H;
@@ -146,6 +157,12 @@ __global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloa
     } else {
       rk[m] = rv[m] = make_uint4(0, 0, 0, 0);
     }
+  }
+  if (kQuant) {   // the FP8 path: K codes and the block's scale, max |V| into the head's maximum
+    const float mk = block_absmax(rk, qred);
+    quant_block_rows(rk, mk, f8.k8, f8.sk + (size_t)bh * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
+    const float mv = block_absmax(rv, qred);
+    if (tid == 0) atomicMax(f8.vmax + bh, __float_as_uint(mv));
   }
   // ---- block mean of the keys
   {
@@ -272,10 +289,16 @@ __global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloa
 }
 
 void launch_sol2_summaries(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                           const Work& w, cudaStream_t st) {
-  summary_q_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, s, w);
+                           const Work& w, cudaStream_t st, const Fp8Work* f8) {
+  if (f8)
+    summary_q_kernel<true><<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, s, w, *f8);
+  else
+    summary_q_kernel<false><<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, s, w, Fp8Work{});
   qdir_kernel<<<s.BH, 8 * kHeadDim, 0, st>>>(s, w);
-  summary_kv_groups_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(k, v, s, w);
+  if (f8)
+    summary_kv_groups_kernel<true><<<dim3(s.Nb, s.BH), 256, 0, st>>>(k, v, s, w, *f8);
+  else
+    summary_kv_groups_kernel<false><<<dim3(s.Nb, s.BH), 256, 0, st>>>(k, v, s, w, Fp8Work{});
 }
 
 }  // namespace sol

@@ -7,6 +7,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "fp8.cuh"
 
 namespace sol {
 
@@ -17,11 +18,15 @@ namespace sol {
 // Outputs per (b, h, j): Qbar, Kbar (FP32 means over the valid tokens), BF16 copies of Kbar and
 // of the value mean Vbar (surrogate MMA operands), and optionally the two 32-token anchor means of Q.
 // -------------------------------------------------------------------------------------------------
+// With kQuant (the FP8 path), the same pass also quantises Q and K per block (fp8.cuh,
+// quant_block_rows) and folds the block's max |V| into the head's maximum.
+template <bool kQuant>
 __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __restrict__ q,
                                                       const __nv_bfloat16* __restrict__ k,
                                                       const __nv_bfloat16* __restrict__ v, Shape s, Work w,
-                                                      int anchors) {
+                                                      int anchors, Fp8Work f8) {
   __shared__ float red[8][4][kHeadDim];
+  __shared__ float qred[8];
   const int j = blockIdx.x, b = blockIdx.y / s.H, h = blockIdx.y % s.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c16 = tid & 15, rg = tid >> 4;
@@ -45,6 +50,15 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
       } else {
         rq[m] = rk[m] = rv[m] = make_uint4(0, 0, 0, 0);
       }
+    }
+    if (kQuant) {
+      const size_t bhj = ((size_t)b * s.H + h) * s.Nb + j;
+      const float mq = block_absmax(rq, qred);
+      quant_block_rows(rq, mq, f8.q8, f8.sq + bhj, s.N, s.H, b, h, t0, n, tid);
+      const float mk = block_absmax(rk, qred);
+      quant_block_rows(rk, mk, f8.k8, f8.sk + bhj, s.N, s.H, b, h, t0, n, tid);
+      const float mv = block_absmax(rv, qred);
+      if (tid == 0) atomicMax(f8.vmax + (size_t)b * s.H + h, __float_as_uint(mv));
     }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -340,8 +354,11 @@ void launch_dense_mask(const Shape& s, const Work& w, int qb_lo, int qb_hi, cuda
 }
 
 void launch_summary(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const Shape& s,
-                    const Work& w, bool anchors, cudaStream_t st) {
-  summary_kernel<<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, k, v, s, w, anchors ? 1 : 0);
+                    const Work& w, bool anchors, cudaStream_t st, const Fp8Work* f8) {
+  if (f8)
+    summary_kernel<true><<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, k, v, s, w, anchors ? 1 : 0, *f8);
+  else
+    summary_kernel<false><<<dim3(s.Nb, s.BH), 256, 0, st>>>(q, k, v, s, w, anchors ? 1 : 0, Fp8Work{});
 }
 
 void launch_kstats(const Shape& s, const Work& w, cudaStream_t st) {
