@@ -21,9 +21,10 @@
 //    column (P of a warpgroup: 64 keys in 16 columns), gathered by byte permutes.  No exponential,
 //    no row sum on the CUDA cores.  The kernel is bound by this instruction stream, not by the
 //    tensor cores: the paired lanes and permutes took it from 10.2 to 9.2 ms at 64K x 32 heads.
-//  * Row sums: for every P product a second one with N = 16 against a block of E4M3 ones
-//    accumulates the sum of the decoded weights in TMEM (L_w), so the denominator is exactly the
-//    FP32 sum of the weights the P V product used; it is rescaled with O when the pivot moves.
+//  * Row sums: the P V product runs with N = 144, its B operand's channels 128..143 being E4M3 ones,
+//    so the same instruction accumulates the sum of the decoded weights in TMEM (L_w) beside O_w:
+//    the denominator is exactly the FP32 sum of the weights the P V product used (sums of E4M3
+//    weights are exact in FP32 at these sizes); it is rescaled with O when the pivot moves.
 //  * Pivot: an integer in base 2, moved only when the running maximum exceeds it by more than 8, to
 //    ceil(max) - 8 (every coded score then has u <= 8, so the clip at 120 never acts); rescale
 //    factors are exact powers of two.
@@ -44,9 +45,9 @@ constexpr int kDescRing = 8;                // tile descriptors in flight
 constexpr uint32_t kTile8 = 128 * 128;      // 128 rows x 128 E4M3 channels (16 KB), one swizzled tile
 constexpr uint32_t kBox8 = 64 * 128;        // one 64-row box (8 KB)
 // TMEM columns: S (128 x 128 FP32); P double buffer (per buffer 32 columns: warpgroup w's 64 keys
-// as E4M3 codes in columns 16 w .. 16 w + 15); L_w (row sums, 16 columns each, column 0 read);
-// O_w (128 columns each).
-constexpr uint32_t kColS = 0, kColP = 128, kColL = 192, kColO = 256;
+// as E4M3 codes in columns 16 w .. 16 w + 15); per warpgroup one N = 144 accumulator at
+// kColO + kOStride w: O_w in its first 128 columns and the row sum L_w in the next 16 (all equal).
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kOStride = 160;
 
 enum : uint32_t { kTilePair = 0, kTileSingle = 1, kTilePooled = 2 };
 
@@ -61,7 +62,7 @@ struct __align__(1024) Fp8Smem {
   uint8_t q[kTile8];               // 128 query rows x 128 channels, K-major SW128
   uint8_t k[kStages][kTile8];      // 128 keys x 128 channels, K-major SW128
   uint8_t v[kStages][kTile8];      // 128 keys x 128 channels: MN-major SW128 B operand of P V
-  uint8_t ones[16 * 128];          // E4M3 1.0 (0x38): B operand of the row-sum product
+  uint8_t ones[32 * 128];          // E4M3 1.0 (0x38): channels 128..143 of the P V product's B operand
   TileDesc8 desc[kDescRing];
   uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
   uint64_t dfull[kDescRing];
@@ -122,15 +123,22 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-// Four ExpCast codes packed first-key-lowest, bit for bit those of expcast_code_f32 / pack_codes4:
-// the same FMA, clamp and 1.5 * 2^23 add (paired lanes of f32x2 instructions round as the scalar
-// ones do), then the low bytes gathered by three byte permutes.
-__device__ __forceinline__ uint32_t expcast_pack4(float x0, float x1, float x2, float x3, uint64_t f8_2, uint64_t c0_2) {
-  const uint64_t magic2 = f2(12582912.0f, 12582912.0f);
-  float2 a = unf2(fma2(f2(x0, x1), f8_2, c0_2));
-  float2 b = unf2(fma2(f2(x2, x3), f8_2, c0_2));
-  const float2 ra = unf2(add2(f2(fmaxf(a.x, 0.0f), fmaxf(a.y, 0.0f)), magic2));
-  const float2 rb = unf2(add2(f2(fmaxf(b.x, 0.0f), fmaxf(b.y, 0.0f)), magic2));
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Four ExpCast codes packed first-key-lowest, bit for bit those of expcast_code_f32 / pack_codes4.
+// The caller passes f8 / 128 and c0 / 128: scaling by a power of two commutes with rounding, so the
+// saturating FMA yields max(RN(x f8 + c0), 0) / 128 and does the clamp at 0 in the same
+// instruction (codes stay below 128: the pivot rule keeps u <= 8, so y <= 119.65).  Adding
+// 1.5 * 2^16 (unit in the last place 2^-7) on f32x2 lanes rounds 128 y' to the nearest even
+// integer in the low bits; three byte permutes gather the four low bytes.
+__device__ __forceinline__ uint32_t expcast_pack4(float x0, float x1, float x2, float x3, float f8s, float c0s) {
+  const uint64_t magic2 = f2(98304.0f, 98304.0f);
+  const float2 ra = unf2(add2(f2(fma_sat(x0, f8s, c0s), fma_sat(x1, f8s, c0s)), magic2));
+  const float2 rb = unf2(add2(f2(fma_sat(x2, f8s, c0s), fma_sat(x3, f8s, c0s)), magic2));
   const uint32_t lo = prmt(__float_as_uint(ra.x), __float_as_uint(ra.y), 0x0040u);
   const uint32_t hi = prmt(__float_as_uint(rb.x), __float_as_uint(rb.y), 0x0040u);
   return prmt(lo, hi, 0x5410u);
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(384, 1)
   }
   {
     uint32_t* ones = reinterpret_cast<uint32_t*>(sm.ones);
-    for (int i = tid; i < 16 * 128 / 4; i += 384) ones[i] = 0x38383838u;
+    for (int i = tid; i < 32 * 128 / 4; i += 384) ones[i] = 0x38383838u;
     fence_async_smem();   // generic-proxy writes, read by the tensor cores
   }
   if (warp == 1) {
@@ -344,8 +352,10 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       bool ok = true;
       bool b_started = false;
-      const uint32_t idesc_pv = idesc_e4m3(128, 128, false, true);
-      const uint32_t idesc_l = idesc_e4m3(128, 16, false, false);
+      // N = 144: channels 0..127 are V, channels 128..143 a second 128-byte atom of the MN-major
+      // operand, placed (by its leading byte offset) on a block of E4M3 ones, so the product's last 16
+      // columns accumulate the row sums of the decoded weights in the same instruction
+      const uint32_t idesc_pv = idesc_e4m3(128, 144, false, true);
       const uint32_t ones_base = smem_u32(&sm.ones[0]);
       for (int u = 0; ok; ++u) {
         const int s = u % kStages;
@@ -368,11 +378,10 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t p_col = tmem + kColP + 32 * bsel + 16 * w;   // P_w: 64 keys in 16 columns
             for (int kk = 0; kk < 2; ++kk) {
               // keys 64 w + 32 kk .. + 31: four 8-row groups of the MN-major V tile
-              const uint64_t bd = sdesc_sw128(v_base + w * kBox8 + kk * 4096, kTile8, 1024);
+              const uint32_t vs = v_base + w * kBox8 + kk * 4096;
+              const uint64_t bd = sdesc_sw128(vs, ones_base - vs, 1024);
               const bool acc = w == 0 ? (u > 0 || kk > 0) : (b_started || kk > 0);
-              umma_ts_f8(tmem + kColO + 128 * w, p_col + 8 * kk, bd, idesc_pv, acc ? 1u : 0u);
-              umma_ts_f8(tmem + kColL + 16 * w, p_col + 8 * kk, sdesc_sw128(ones_base + 32 * kk, 16, 1024), idesc_l,
-                         acc ? 1u : 0u);
+              umma_ts_f8(tmem + kColO + kOStride * w, p_col + 8 * kk, bd, idesc_pv, acc ? 1u : 0u);
             }
             if (w == 1) b_started = true;
           }
@@ -430,8 +439,8 @@ __global__ void __launch_bounds__(384, 1)
     const int tok = 64 * qb0 + r;
     const bool row_valid = tok >= p.row_lo && tok < p.row_hi;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    const uint32_t o_addr = lane_addr + kColO + 128 * wg;
-    const uint32_t l_addr = lane_addr + kColL + 16 * wg;
+    const uint32_t o_addr = lane_addr + kColO + kOStride * wg;
+    const uint32_t l_addr = o_addr + 128;
     const uint32_t* mrow = p.mask + ((size_t)bh * p.Nb + min(qi, p.Nb - 1)) * p.Nw;
     const float sq_row = f.sq[(size_t)bh * p.Nb + min(qi, p.Nb - 1)];
     const float fs_row = sq_row * kScale * kLog2e;   // base-2 score per unit of Q8 . K8, before s_K
@@ -479,12 +488,24 @@ __global__ void __launch_bounds__(384, 1)
           const int wd0 = 4 * d.j0 + 2 * wg;
           const uint32_t m_own0 = wd0 < p.Nw ? mrow[wd0] : 0xffffffffu;
           const uint32_t m_own1 = wd0 + 1 < p.Nw ? mrow[wd0 + 1] : 0xffffffffu;
+          if (jb_own + 64 < p.Nb) {
+            // every column a full block other than the last: bias log2 64 throughout
+            const uint64_t fs2 = f2(fs, fs), six2 = f2(6.0f, 6.0f);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int j = jb_own + c;
-            const float bias = (j == p.Nb - 1) ? lg_last : 6.0f;
-            const bool ex = (((c < 32) ? m_own0 : m_own1) >> (c & 31)) & 1u;
-            x[c] = (j < p.Nb && !ex) ? fmaf(x[c], fs, bias) : -INFINITY;
+            for (int c = 0; c < 64; c += 2) {
+              const float2 v = unf2(fma2(f2(x[c], x[c + 1]), fs2, six2));
+              const uint32_t m = (c < 32) ? m_own0 : m_own1;
+              x[c] = ((m >> (c & 31)) & 1u) ? -INFINITY : v.x;
+              x[c + 1] = ((m >> ((c + 1) & 31)) & 1u) ? -INFINITY : v.y;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const int j = jb_own + c;
+              const float bias = (j == p.Nb - 1) ? lg_last : 6.0f;
+              const bool ex = (((c < 32) ? m_own0 : m_own1) >> (c & 31)) & 1u;
+              x[c] = (j < p.Nb && !ex) ? fmaf(x[c], fs, bias) : -INFINITY;
+            }
           }
         } else if (lim_own < 64) {
 #pragma unroll
@@ -505,11 +526,10 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t pk[16];
       if (lim_own > 0) {
         const float c0 = kExpCastOffset - 8.0f * (pivot == -INFINITY ? 0.f : pivot);
-        const float f8 = pooled ? 8.0f : 8.0f * fs;
-        const uint64_t f8_2 = f2(f8, f8), c0_2 = f2(c0, c0);
+        const float f8s = (pooled ? 8.0f : 8.0f * fs) * 0.0078125f, c0s = c0 * 0.0078125f;
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4)
-          pk[c4] = expcast_pack4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3], f8_2, c0_2);
+          pk[c4] = expcast_pack4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3], f8s, c0s);
       } else {
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) pk[c4] = 0u;
@@ -622,8 +642,8 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       uint32_t oa[64], ob[64];
-      const uint32_t self_addr = lane_addr + kColO + 128 * wg + 64 * wg;
-      const uint32_t other_addr = lane_addr + kColO + 128 * (1 - wg) + 64 * wg;
+      const uint32_t self_addr = lane_addr + kColO + kOStride * wg + 64 * wg;
+      const uint32_t other_addr = lane_addr + kColO + kOStride * (1 - wg) + 64 * wg;
       tmem_ld32_at<0>(self_addr, oa);
       tmem_ld32_at<32>(self_addr + 32, oa);
       tmem_ld32_at<0>(other_addr, ob);
