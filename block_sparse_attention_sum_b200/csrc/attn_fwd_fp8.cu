@@ -16,11 +16,11 @@
 //    E4M3 compressed keys / values (Kbar8, Vbar8) in the same formats.
 //  * Scales: the producer writes the key operand's two 64-row scales into the tile descriptor;
 //    the softmax folds s_Q s_K / sqrt(128) log2 e into one multiplier per row and half-tile.
-//  * Softmax: a score's code is one FMA, a clamp at 0 and an add of 1.5 * 2^23 (its low byte is
-//    the rounded code), the FMA and the add on paired f32x2 lanes; four codes per 32-bit TMEM
-//    column (P of a warpgroup: 64 keys in 16 columns), gathered by byte permutes.  No exponential,
-//    no row sum on the CUDA cores.  The kernel is bound by this instruction stream, not by the
-//    tensor cores: the paired lanes and permutes took it from 10.2 to 9.2 ms at 64K x 32 heads.
+//  * Softmax: a score's code is one saturating FMA (on the score scaled by 2^-7, so the
+//    saturation is the clamp at 0) and an add of 1.5 * 2^16 on paired f32x2 lanes, whose low byte
+//    is the rounded code; four codes per 32-bit TMEM column (P of a warpgroup: 64 keys in 16
+//    columns), gathered by byte permutes.  No exponential, no row sum on the CUDA cores.  The
+//    kernel is bound by this instruction stream, not by the tensor cores.
 //  * Row sums: the P V product runs with N = 144, its B operand's channels 128..143 being E4M3 ones,
 //    so the same instruction accumulates the sum of the decoded weights in TMEM (L_w) beside O_w:
 //    the denominator is exactly the FP32 sum of the weights the P V product used (sums of E4M3
