@@ -960,6 +960,15 @@ int sol_attn_expcast_host(const float* x, int n, float fs, float pivot, unsigned
   return SOL_OK;
 }
 
+int sol_attn_quot448_host(const float* x, int n, float m, float* q) {
+  if (!x || !q) return fail(SOL_ERR_NULL, "x and q must be non-NULL");
+  if (n < 0) return fail(SOL_ERR_SHAPE, "n must be non-negative (got %d)", n);
+  if (!(m > 0.f) || !std::isfinite(m)) return fail(SOL_ERR_OPTION, "m must be positive and finite");
+  const Quot448 c = quot448_setup(m);
+  for (int i = 0; i < n; ++i) q[i] = quot448(x[i], c);
+  return SOL_OK;
+}
+
 void sol_attn_set_workspace_limit(size_t bytes) {
   std::lock_guard<std::mutex> lock(g_mu);
   g_ws_limit = bytes;

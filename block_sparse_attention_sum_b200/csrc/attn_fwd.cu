@@ -495,6 +495,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32_at<0>(s_addr, own);
         tmem_ld32_at<32>(s_addr + 32, own);
         tmem_ld_wait();
+        reg_fence(own);
       }
       // S is in registers: the next tile's Q K^T may overwrite it
       tc_fence_before();
@@ -569,6 +570,7 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld32_at<0>(o_addr + 64 * half, o);
           tmem_ld32_at<32>(o_addr + 64 * half + 32, o);
           tmem_ld_wait();
+          reg_fence(o);
 #pragma unroll
           for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
           tmem_st32_at<0>(o_addr + 64 * half, o);
@@ -672,6 +674,8 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld32_at<0>(other_addr, ob);
       tmem_ld32_at<32>(other_addr + 32, ob);
       tmem_ld_wait();
+      reg_fence(oa);
+      reg_fence(ob);
       const float ws = (self_written && w_self > 0.f) ? w_self * scale_o : 0.f;
       const float wo = (other_written && w_other > 0.f) ? w_other * scale_o : 0.f;
       if (p.kv_splits > 1) {

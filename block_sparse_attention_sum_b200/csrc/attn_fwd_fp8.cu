@@ -475,6 +475,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32_at<0>(s_addr, own);
         tmem_ld32_at<32>(s_addr + 32, own);
         tmem_ld_wait();
+        reg_fence(own);
       }
       tc_fence_before();
       mbar_arrive(&sm.sread);
@@ -552,13 +553,15 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld32_at<0>(o_addr + 64 * half, o);
           tmem_ld32_at<32>(o_addr + 64 * half + 32, o);
           tmem_ld_wait();
+          reg_fence(o);
 #pragma unroll
           for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * fa);
           tmem_st32_at<0>(o_addr + 64 * half, o);
           tmem_st32_at<32>(o_addr + 64 * half + 32, o);
         }
-        const uint32_t lv = tmem_ld1(l_addr);
+        uint32_t lv = tmem_ld1(l_addr);
         tmem_ld_wait();
+        reg_fence1(lv);
         tmem_st1(l_addr, __float_as_uint(__uint_as_float(lv) * fa));
       }
       tmem_st_wait();
@@ -572,8 +575,9 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     float l = 0.f;
     {
-      const uint32_t lv = tmem_ld1(l_addr);
+      uint32_t lv = tmem_ld1(l_addr);
       tmem_ld_wait();
+      reg_fence1(lv);
       if (pivot != -INFINITY) l = __uint_as_float(lv);
     }
     // exchange (pivot, l) with the other warpgroup's thread of this row and merge:
@@ -649,6 +653,8 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld32_at<0>(other_addr, ob);
       tmem_ld32_at<32>(other_addr + 32, ob);
       tmem_ld_wait();
+      reg_fence(oa);
+      reg_fence(ob);
       const float ws = (self_written && w_self > 0.f) ? w_self * scale_o : 0.f;
       const float wo = (other_written && w_other > 0.f) ? w_other * scale_o : 0.f;
       if (row_valid) {

@@ -56,6 +56,54 @@ __host__ __device__ __forceinline__ float pow2i(float k) {
   return r;
 }
 
+// X / s for s = m / 448 (m = max |X| > 0 of the scale's group), as the quantisers evaluate it:
+// RN(RN(x * 448) / m) without a division per element.  With s2 = 2^(127 - E) (E the biased
+// exponent of m) scaling changes no rounding, so the value is RN(a / m2) for a = RN(x * 448 s2)
+// and m2 = m s2 in [1, 2).  With y = RN(1 / m2), q = RN(a y) lies within one unit in the last place
+// of a / m2, the remainder a - q m2 is exact in one FMA, and RN(q + (a - q m2) y) is the correctly
+// rounded quotient (Markstein's theorem, the correction step of the IA-64 division sequences).
+// Outside 2^-100 <= m < 2^101 the division is taken as written.  The sign is copied from x, so
+// -0 stays -0 as in the division.
+struct Quot448 {
+  float k448;   // 448 s2
+  float m2;     // m s2
+  float y;      // RN(1 / m2)
+  float m;      // m itself, for the division outside the range
+  bool fast;
+};
+
+__host__ __device__ __forceinline__ Quot448 quot448_setup(float m) {
+  uint32_t bits;
+#ifdef __CUDA_ARCH__
+  bits = __float_as_uint(m);
+#else
+  __builtin_memcpy(&bits, &m, 4);
+#endif
+  const uint32_t eb = (bits >> 23) & 0xffu;
+  Quot448 c;
+  c.m = m;
+  c.fast = eb >= 27u && eb <= 227u;
+  const uint32_t sbits = (254u - (c.fast ? eb : 127u)) << 23;   // 2^(127 - E)
+  float s2;
+#ifdef __CUDA_ARCH__
+  s2 = __uint_as_float(sbits);
+#else
+  __builtin_memcpy(&s2, &sbits, 4);
+#endif
+  c.k448 = 448.0f * s2;
+  c.m2 = m * s2;
+  c.y = 1.0f / c.m2;
+  return c;
+}
+
+__host__ __device__ __forceinline__ float quot448(float x, const Quot448& c) {
+  if (!c.fast) return (x * 448.0f) / c.m;
+  const float a = x * c.k448;
+  const float q = a * c.y;
+  const float r = fmaf(-q, c.m2, a);
+  return copysignf(fmaf(r, c.y, q), x);
+}
+
 // Pivot rule of the online softmax: the pivot is an integer (base 2) and moves only when the running
 // maximum exceeds it by more than 8, to ceil(max) - 8, so that every coded score satisfies u <= 8.
 // Returns the new pivot; *alpha = 2^(old - new) rescales what was accumulated against the old one
@@ -129,25 +177,49 @@ __device__ __forceinline__ uint32_t to_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// X / s with s = m / 448, evaluated as (x * 448) / m: for a BF16 x the product is exact and the
-// quotient is correctly rounded, so a value that lies exactly halfway between two E4M3 numbers
+// X / s is evaluated as (x * 448) / m (quot448): for a BF16 x the product is exact and the
+// quotient correctly rounded, so a value that lies exactly halfway between two E4M3 numbers
 // (frequent: x and m share most of their few mantissa bits) stays exactly halfway and rounds to
 // even, as the definition asks; x / fl(m / 448) can land just off the midpoint and round the
-// other way.  m > 0.
-__device__ __forceinline__ float scaled448(float x, float m) { return (x * 448.0f) / m; }
+// other way.
 
-// Eight values of a block with maximum |X| = m > 0, as four E4M3 pairs in one 8-byte word.
-__device__ __forceinline__ uint2 codes8(const float (&v)[8], float m) {
+// quot448 of two values on f32x2 lanes (each lane rounds as the scalar instruction does, so the
+// pair equals two quot448 calls bit for bit); c.fast must hold.
+__device__ __forceinline__ float2 quot448x2(float x0, float x1, const Quot448& c) {
+  uint64_t x, k, y, m2, a, q, r, o;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(k) : "f"(c.k448));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(y) : "f"(c.y));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(m2) : "f"(-c.m2));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(a) : "l"(x), "l"(k));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q) : "l"(a), "l"(y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(q), "l"(m2), "l"(a));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(o) : "l"(r), "l"(y), "l"(q));
+  float2 res;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(res.x), "=f"(res.y) : "l"(o));
+  return make_float2(copysignf(res.x, x0), copysignf(res.y, x1));
+}
+
+// Eight values of a block with maximum |X| = m > 0 (c = quot448_setup(m)), as four E4M3 pairs in
+// one 8-byte word.
+__device__ __forceinline__ uint2 codes8(const float (&v)[8], const Quot448& c) {
   uint32_t w[4];
+  if (c.fast) {
 #pragma unroll
-  for (int e = 0; e < 4; ++e) w[e] = to_e4m3x2(scaled448(v[2 * e], m), scaled448(v[2 * e + 1], m));
+    for (int e = 0; e < 4; ++e) {
+      const float2 q = quot448x2(v[2 * e], v[2 * e + 1], c);
+      w[e] = to_e4m3x2(q.x, q.y);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w[e] = to_e4m3x2(quot448(v[2 * e], c), quot448(v[2 * e + 1], c));
+  }
   return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
-// The largest |x| of a 64-token block held by 256 threads (each holds four rows of 8 BF16 channels,
-// `rows`, as the block-summary kernels load them): warp shuffles, then eight warp maxima through
-// `red` (8 floats of shared memory; the call synchronises the block twice).
-__device__ __forceinline__ float block_absmax(const uint4 (&rows)[4], float* red) {
+// This thread's largest |x| over its four rows of 8 BF16 channels (`rows`, as the block-summary
+// kernels load them).
+__device__ __forceinline__ float thread_absmax(const uint4 (&rows)[4]) {
   float m = 0.f;
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
@@ -158,15 +230,32 @@ __device__ __forceinline__ float block_absmax(const uint4 (&rows)[4], float* red
       m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
     }
   }
+  return m;
+}
+
+// Block-wide maxima (256 threads) of kT per-thread values, all in one pass: warp shuffles, then the
+// eight warp maxima of each value through `red` (8 kT floats of shared memory); the call
+// synchronises the block twice whatever kT.
+template <int kT>
+__device__ __forceinline__ void block_max(float (&m)[kT], float* red) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  float b = red[0];
+  for (int t = 0; t < kT; ++t) {
 #pragma unroll
-  for (int i = 1; i < 8; ++i) b = fmaxf(b, red[i]);
+    for (int o = 16; o > 0; o >>= 1) m[t] = fmaxf(m[t], __shfl_xor_sync(0xffffffffu, m[t], o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int t = 0; t < kT; ++t) red[8 * t + (threadIdx.x >> 5)] = m[t];
+  }
   __syncthreads();
-  return b;
+#pragma unroll
+  for (int t = 0; t < kT; ++t) {
+    float b = red[8 * t];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) b = fmaxf(b, red[8 * t + i]);
+    m[t] = b;
+  }
+  __syncthreads();
 }
 
 // E4M3 codes of one 64-token block (one scale, s = max |X| / 448; an all-zero block keeps s = 1 and
@@ -177,6 +266,7 @@ __device__ __forceinline__ void quant_block_rows(const uint4 (&rows)[4], float m
                                                  int H, int b, int h, int t0, int n, int tid) {
   const int c16 = tid & 15, rg = tid >> 4;
   if (tid == 0) *scale = m > 0.f ? m / 448.0f : 1.0f;
+  const Quot448 qc = quot448_setup(m > 0.f ? m : 1.0f);
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int row = rg + 16 * r;
@@ -190,7 +280,7 @@ __device__ __forceinline__ void quant_block_rows(const uint4 (&rows)[4], float m
       v[2 * e + 1] = f.y;
     }
     *reinterpret_cast<uint2*>(x8 + (((size_t)b * N + t0 + row) * H + h) * 128 + 8 * c16) =
-        m > 0.f ? codes8(v, m) : make_uint2(0u, 0u);
+        m > 0.f ? codes8(v, qc) : make_uint2(0u, 0u);
   }
 }
 #endif  // __CUDACC__

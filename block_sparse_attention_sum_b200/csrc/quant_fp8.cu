@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const __nv_bfloat16* __res
   const float m = __uint_as_float(vmax[bh]);
   const float sc = m > 0.f ? m / 448.0f : 1.0f;
   if (j == 0 && tid == 0) sv[bh] = sc;
+  const Quot448 qc = quot448_setup(m > 0.f ? m : 1.0f);
   float vals[4][8], amax;
   load_rows_bf16(v, s, b, h, t0, n, tid, vals, &amax);
   const int c16 = tid & 15, rg = tid >> 4;
@@ -75,7 +76,7 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const __nv_bfloat16* __res
     const int row = rg + 16 * r;
     if (row < n)
       *reinterpret_cast<uint2*>(v8 + (((size_t)b * s.N + t0 + row) * s.H + h) * kHeadDim + 8 * c16) =
-          m > 0.f ? codes8(vals[r], m) : make_uint2(0u, 0u);
+          m > 0.f ? codes8(vals[r], qc) : make_uint2(0u, 0u);
   }
   // column sums: rows beyond n were loaded as zeros
 #pragma unroll
@@ -89,7 +90,7 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const __nv_bfloat16* __res
       a1 += colsum[g][2 * tid + 1];
     }
     const float inv_n = 1.0f / (float)n;
-    const uint32_t w = m > 0.f ? to_e4m3x2(scaled448(a0 * inv_n, m), scaled448(a1 * inv_n, m)) : 0u;
+    const uint32_t w = m > 0.f ? to_e4m3x2(quot448(a0 * inv_n, qc), quot448(a1 * inv_n, qc)) : 0u;
     *reinterpret_cast<uint16_t*>(vbar8 + ((size_t)bh * Nbp + j) * kHeadDim + 2 * tid) = (uint16_t)w;
   }
 }
@@ -121,11 +122,12 @@ __global__ void __launch_bounds__(256) quant_kbar_kernel(const float* __restrict
   const float m = block_max_256(amax, red);
   const float sc = m > 0.f ? m / 448.0f : 1.0f;
   if (tid == 0) skbar[(size_t)bh * (Nbp / 64) + g] = sc;
+  const Quot448 qc = quot448_setup(m > 0.f ? m : 1.0f);
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int j = 64 * g + rg + 16 * r;
     const size_t off = ((size_t)bh * Nbp + j) * kHeadDim + 8 * c16;
-    *reinterpret_cast<uint2*>(kbar8 + off) = (j < s.Nb && m > 0.f) ? codes8(vals[r], m) : make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(kbar8 + off) = (j < s.Nb && m > 0.f) ? codes8(vals[r], qc) : make_uint2(0u, 0u);
     if (j >= s.Nb) *reinterpret_cast<uint2*>(vbar8 + off) = make_uint2(0u, 0u);
   }
 }

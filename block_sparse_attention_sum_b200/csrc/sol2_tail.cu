@@ -68,8 +68,9 @@ __global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __r
                   : make_uint4(0, 0, 0, 0);
   }
   if (kQuant) {   // the FP8 path: Q codes and the block's scale in the same pass
-    const float mq = block_absmax(rq, qred);
-    quant_block_rows(rq, mq, f8.q8, f8.sq + ((size_t)b * s.H + h) * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
+    float mq[1] = {thread_absmax(rq)};
+    block_max(mq, qred);
+    quant_block_rows(rq, mq[0], f8.q8, f8.sq + ((size_t)b * s.H + h) * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
   }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloa
                                                                 const __nv_bfloat16* __restrict__ v, Shape s, Work w,
                                                                 Fp8Work f8) {
   __shared__ float red[8][4][kHeadDim];
-  __shared__ float qred[8];
+  __shared__ float qred[2 * 8];
   __shared__ float kbar_s[kHeadDim];
   __shared__ int n1_s;
   const int j = blockIdx.x, bh = blockIdx.y, b = bh / s.H, h = bh % s.H;
@@ -159,10 +160,10 @@ __global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloa
     }
   }
   if (kQuant) {   // the FP8 path: K codes and the block's scale, max |V| into the head's maximum
-    const float mk = block_absmax(rk, qred);
-    quant_block_rows(rk, mk, f8.k8, f8.sk + (size_t)bh * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
-    const float mv = block_absmax(rv, qred);
-    if (tid == 0) atomicMax(f8.vmax + bh, __float_as_uint(mv));
+    float mx[2] = {thread_absmax(rk), thread_absmax(rv)};
+    block_max(mx, qred);
+    quant_block_rows(rk, mx[0], f8.k8, f8.sk + (size_t)bh * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
+    if (tid == 0) atomicMax(f8.vmax + bh, __float_as_uint(mx[1]));
   }
   // ---- block mean of the keys
   {

@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
                                                       const __nv_bfloat16* __restrict__ v, Shape s, Work w,
                                                       int anchors, Fp8Work f8) {
   __shared__ float red[8][4][kHeadDim];
-  __shared__ float qred[8];
+  __shared__ float qred[3 * 8];
   const int j = blockIdx.x, b = blockIdx.y / s.H, h = blockIdx.y % s.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c16 = tid & 15, rg = tid >> 4;
@@ -53,12 +53,11 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
     }
     if (kQuant) {
       const size_t bhj = ((size_t)b * s.H + h) * s.Nb + j;
-      const float mq = block_absmax(rq, qred);
-      quant_block_rows(rq, mq, f8.q8, f8.sq + bhj, s.N, s.H, b, h, t0, n, tid);
-      const float mk = block_absmax(rk, qred);
-      quant_block_rows(rk, mk, f8.k8, f8.sk + bhj, s.N, s.H, b, h, t0, n, tid);
-      const float mv = block_absmax(rv, qred);
-      if (tid == 0) atomicMax(f8.vmax + (size_t)b * s.H + h, __float_as_uint(mv));
+      float mx[3] = {thread_absmax(rq), thread_absmax(rk), thread_absmax(rv)};
+      block_max(mx, qred);
+      quant_block_rows(rq, mx[0], f8.q8, f8.sq + bhj, s.N, s.H, b, h, t0, n, tid);
+      quant_block_rows(rk, mx[1], f8.k8, f8.sk + bhj, s.N, s.H, b, h, t0, n, tid);
+      if (tid == 0) atomicMax(f8.vmax + (size_t)b * s.H + h, __float_as_uint(mx[2]));
     }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {

@@ -45,6 +45,7 @@ EXPORTS = [
     "sol_attn_fwd_fp8",
     "sol_attn2_fwd_fp8",
     "sol_attn_expcast_host",
+    "sol_attn_quot448_host",
 ]
 
 STATUS = {
@@ -170,6 +171,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sol_attn2_fwd_fp8.restype = i
     lib.sol_attn_expcast_host.argtypes = [ctypes.POINTER(ctypes.c_float), i, f, f, ctypes.POINTER(ctypes.c_uint)]
     lib.sol_attn_expcast_host.restype = i
+    lib.sol_attn_quot448_host.argtypes = [ctypes.POINTER(ctypes.c_float), i, f, ctypes.POINTER(ctypes.c_float)]
+    lib.sol_attn_quot448_host.restype = i
     _lib = lib
     return lib
 
@@ -301,6 +304,20 @@ def expcast_host(x, fs: float, pivot: float):
                                    float(pivot), words.ctypes.data_as(ctypes.POINTER(ctypes.c_uint)))
     _check(rc)
     return words.view(np.uint8).copy()
+
+
+def quot448_host(x, m: float):
+    """The FP8 quantisers' scaled value x * 448 / m (before the E4M3 rounding) evaluated on the host
+    by the kernels' own inline function: float32 array of len(x)."""
+    import numpy as np
+
+    xs = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    q = np.empty_like(xs)
+    lib = load_library()
+    rc = lib.sol_attn_quot448_host(xs.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), int(xs.size), float(m),
+                                   q.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    _check(rc)
+    return q
 
 
 def sol_attn_fwd_varlen(q, k, v, cu_seqlens, tau=1.0, sink_start=-1, sink_tokens=0, out=None, stream=None,

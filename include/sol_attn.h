@@ -369,6 +369,17 @@ int sol_attn2_fwd_fp8(const void* q, const void* k, const void* v, void* out, in
  */
 int sol_attn_expcast_host(const float* x, int n, float fs, float pivot, unsigned int* words);
 
+/*
+ * Host evaluation of the FP8 quantisers' scaled value X / s, s = m / 448 ([Sol2] "FP8 quantization
+ * and ExpCast": scale = max |X| / 448 of the block or head), as the GPU computes it before the
+ * E4M3 rounding (the same inline function; for checking it without a GPU).  The kernels evaluate
+ * RN(RN(x * 448) / m) without a division per element (a reciprocal per block and one FMA
+ * correction step); this entry point lets a test compare that against the IEEE division.  For n
+ * HOST floats x and 0 < m < inf, q_i = the kernels' value for x_i.  Returns SOL_ERR_NULL,
+ * SOL_ERR_SHAPE (n < 0) or SOL_ERR_OPTION (m) without writing.
+ */
+int sol_attn_quot448_host(const float* x, int n, float m, float* q);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,9 +1,10 @@
 """The FP8 kernels' ExpCast encoder (the inline function their softmax runs, evaluated on the host
-through sol_attn_expcast_host) against the reference's ExpCast codes, and the FP8 entry points'
-host-side argument checks (CPU only).
+through sol_attn_expcast_host) against the reference's ExpCast codes; the quantisers' scaled value
+x * 448 / m (through sol_attn_quot448_host) against the IEEE division it replaces; and the FP8 entry
+points' host-side argument checks (CPU only).
 
 Sol-Attn2 draft, section "FP8 quantization and ExpCast": c(u) = clip_[0,120](RNE(8u + 55.65)) of the
-base-2 score u relative to the pivot."""
+base-2 score u relative to the pivot; codes E4M3(X / s) with s = max |X| / 448."""
 import numpy as np
 import pytest
 
@@ -83,3 +84,51 @@ def test_fp8_entry_points_validate_on_the_host(lib):
         o = sa.Options()
         o.thresh_type = 7
         assert call(fn, opts=ctypes.byref(o)) == -10
+
+
+def _bf16_values(lo_bits, hi_bits):
+    bits = np.arange(lo_bits, hi_bits, dtype=np.uint32) << 16
+    return bits.view(np.float32)
+
+
+def _assert_same_as_division(x, m):
+    import torch
+
+    x = np.asarray(x, dtype=np.float32)
+    with np.errstate(over="ignore"):                        # m near the float32 maximum: x * 448 = inf
+        ref = (x * np.float32(448.0)) / np.float32(m)      # float32: RN(RN(x * 448) / m)
+    got = sa.quot448_host(x, m)
+    tiny = np.abs(ref) < 2.0 ** -20                          # E4M3 code +-0 either way (below 2^-10)
+    assert np.array_equal(got[~tiny].view(np.uint32), ref[~tiny].view(np.uint32)), m
+    assert (np.abs(got[tiny]) < 2.0 ** -20).all() and np.array_equal(np.signbit(got), np.signbit(ref))
+    codes = lambda a: torch.from_numpy(a).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes(got), codes(ref))
+
+
+def test_quantiser_quotient_equals_the_division_for_bf16_blocks(lib):
+    # every BF16 x with |x| <= m, both signs, for block maxima m across the exponent range (the
+    # reciprocal path covers 2^-100 <= m < 2^101, the division is kept outside it)
+    g = np.random.default_rng(3)
+    ms = list(_bf16_values(0x0001, 0x7F80)[g.integers(0, 0x7F7F, 160)])
+    ms += [2.0 ** -100, 2.0 ** -100 * 0.99, 2.0 ** 100, 2.0 ** 101, 3.875, 1.0, 448.0, 1e-30, 3e38]
+    for m in ms:
+        m = float(np.float32(m))
+        mb = int(np.array([m], dtype=np.float32).view(np.uint32)[0] >> 16)
+        x = _bf16_values(0, mb + 1)
+        x = x[np.abs(x) <= m]
+        _assert_same_as_division(np.concatenate([x, -x]), m)
+
+
+def test_quantiser_quotient_equals_the_division_for_fp32_values(lib):
+    # FP32 inputs (the compressed keys' and values' means) at random magnitudes below m
+    g = np.random.default_rng(4)
+    for m in np.float32(2.0) ** g.uniform(-60, 60, 200).astype(np.float32) * g.uniform(1, 2, 200).astype(np.float32):
+        x = (g.uniform(-1, 1, 5000) * np.float32(2.0) ** g.uniform(-30, 0, 5000)).astype(np.float32) * m
+        _assert_same_as_division(x, float(m))
+
+
+def test_quantiser_quotient_keeps_exact_midpoints_and_signed_zero(lib):
+    # 2.90625 * 448 / 3.875 = 336, halfway between the E4M3 values 320 and 352: must stay exact
+    q = sa.quot448_host([2.90625, -2.90625, 0.0, -0.0, 3.875], 3.875)
+    assert q[0] == 336.0 and q[1] == -336.0 and q[4] == 448.0
+    assert q[2] == 0.0 and not np.signbit(q[2]) and q[3] == 0.0 and np.signbit(q[3])
