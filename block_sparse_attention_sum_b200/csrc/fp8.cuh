@@ -234,10 +234,11 @@ __device__ __forceinline__ float thread_absmax(const uint4 (&rows)[4]) {
 }
 
 // Block-wide maxima (256 threads) of kT per-thread values, all in one pass: warp shuffles, then the
-// eight warp maxima of each value through `red` (8 kT floats of shared memory); the call
+// eight warp maxima of each value through `red` (8 kT floats of shared memory).  The two halves
+// let a kernel share the block synchronisation between them with other reductions; block_max
 // synchronises the block twice whatever kT.
 template <int kT>
-__device__ __forceinline__ void block_max(float (&m)[kT], float* red) {
+__device__ __forceinline__ void block_max_post(float (&m)[kT], float* red) {
 #pragma unroll
   for (int t = 0; t < kT; ++t) {
 #pragma unroll
@@ -247,7 +248,9 @@ __device__ __forceinline__ void block_max(float (&m)[kT], float* red) {
 #pragma unroll
     for (int t = 0; t < kT; ++t) red[8 * t + (threadIdx.x >> 5)] = m[t];
   }
-  __syncthreads();
+}
+template <int kT>
+__device__ __forceinline__ void block_max_collect(float (&m)[kT], const float* red) {
 #pragma unroll
   for (int t = 0; t < kT; ++t) {
     float b = red[8 * t];
@@ -255,6 +258,12 @@ __device__ __forceinline__ void block_max(float (&m)[kT], float* red) {
     for (int i = 1; i < 8; ++i) b = fmaxf(b, red[8 * t + i]);
     m[t] = b;
   }
+}
+template <int kT>
+__device__ __forceinline__ void block_max(float (&m)[kT], float* red) {
+  block_max_post(m, red);
+  __syncthreads();
+  block_max_collect(m, red);
   __syncthreads();
 }
 

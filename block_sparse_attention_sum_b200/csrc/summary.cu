@@ -51,13 +51,14 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
         rq[m] = rk[m] = rv[m] = make_uint4(0, 0, 0, 0);
       }
     }
+    // FP8 path: the block maxima of |Q|, |K|, |V| share the block synchronisation of the sums; Q and
+    // K are quantised after the sums, once V's registers are free
+    float mx[3];
     if (kQuant) {
-      const size_t bhj = ((size_t)b * s.H + h) * s.Nb + j;
-      float mx[3] = {thread_absmax(rq), thread_absmax(rk), thread_absmax(rv)};
-      block_max(mx, qred);
-      quant_block_rows(rq, mx[0], f8.q8, f8.sq + bhj, s.N, s.H, b, h, t0, n, tid);
-      quant_block_rows(rk, mx[1], f8.k8, f8.sk + bhj, s.N, s.H, b, h, t0, n, tid);
-      if (tid == 0) atomicMax(f8.vmax + (size_t)b * s.H + h, __float_as_uint(mx[2]));
+      mx[0] = thread_absmax(rq);
+      mx[1] = thread_absmax(rk);
+      mx[2] = thread_absmax(rv);
+      block_max_post(mx, qred);
     }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -134,6 +135,13 @@ __global__ void __launch_bounds__(256) summary_kernel(const __nv_bfloat16* __res
           w.qanchor_h[a0 + kHeadDim] = __float2bfloat16_rn(ahi);
         }
       }
+    }
+    if (kQuant) {
+      block_max_collect(mx, qred);
+      const size_t bhj = ((size_t)b * s.H + h) * s.Nb + j;
+      quant_block_rows(rq, mx[0], f8.q8, f8.sq + bhj, s.N, s.H, b, h, t0, n, tid);
+      quant_block_rows(rk, mx[1], f8.k8, f8.sk + bhj, s.N, s.H, b, h, t0, n, tid);
+      if (tid == 0) atomicMax(f8.vmax + (size_t)b * s.H + h, __float_as_uint(mx[2]));
     }
   }
 }
