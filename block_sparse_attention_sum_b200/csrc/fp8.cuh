@@ -234,9 +234,8 @@ __device__ __forceinline__ float thread_absmax(const uint4 (&rows)[4]) {
 }
 
 // Block-wide maxima (256 threads) of kT per-thread values, all in one pass: warp shuffles, then the
-// eight warp maxima of each value through `red` (8 kT floats of shared memory).  The two halves
-// let a kernel share the block synchronisation between them with other reductions; block_max
-// synchronises the block twice whatever kT.
+// eight warp maxima of each value through `red` (8 kT floats of shared memory).  The caller puts a
+// block synchronisation between the two halves, shared with its other reductions.
 template <int kT>
 __device__ __forceinline__ void block_max_post(float (&m)[kT], float* red) {
 #pragma unroll
@@ -258,13 +257,6 @@ __device__ __forceinline__ void block_max_collect(float (&m)[kT], const float* r
     for (int i = 1; i < 8; ++i) b = fmaxf(b, red[8 * t + i]);
     m[t] = b;
   }
-}
-template <int kT>
-__device__ __forceinline__ void block_max(float (&m)[kT], float* red) {
-  block_max_post(m, red);
-  __syncthreads();
-  block_max_collect(m, red);
-  __syncthreads();
 }
 
 // E4M3 codes of one 64-token block (one scale, s = max |X| / 448; an all-zero block keeps s = 1 and

@@ -67,10 +67,12 @@ __global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __r
                                                         8 * c16))
                   : make_uint4(0, 0, 0, 0);
   }
-  if (kQuant) {   // the FP8 path: Q codes and the block's scale in the same pass
-    float mq[1] = {thread_absmax(rq)};
-    block_max(mq, qred);
-    quant_block_rows(rq, mq[0], f8.q8, f8.sq + ((size_t)b * s.H + h) * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
+  // the FP8 path: Q codes and the block's scale in the same pass (the maximum shares the block
+  // synchronisation of the sums)
+  float mq[1];
+  if (kQuant) {
+    mq[0] = thread_absmax(rq);
+    block_max_post(mq, qred);
   }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
@@ -125,6 +127,10 @@ __global__ void __launch_bounds__(256) summary_q_kernel(const __nv_bfloat16* __r
       w.qanchor_h[a0 + kHeadDim] = __float2bfloat16_rn(ahi);
     }
   }
+  if (kQuant) {
+    block_max_collect(mq, qred);
+    quant_block_rows(rq, mq[0], f8.q8, f8.sq + ((size_t)b * s.H + h) * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
+  }
 }
 
 // Key / value pass of the Sol-Attn2 summaries, after the mean query u is known: Kbar (FP32 and the
@@ -159,11 +165,13 @@ __global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloa
       rk[m] = rv[m] = make_uint4(0, 0, 0, 0);
     }
   }
-  if (kQuant) {   // the FP8 path: K codes and the block's scale, max |V| into the head's maximum
-    float mx[2] = {thread_absmax(rk), thread_absmax(rv)};
-    block_max(mx, qred);
-    quant_block_rows(rk, mx[0], f8.k8, f8.sk + (size_t)bh * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
-    if (tid == 0) atomicMax(f8.vmax + bh, __float_as_uint(mx[1]));
+  // the FP8 path: K codes and the block's scale, max |V| into the head's maximum; the maxima share
+  // the block synchronisation of the key mean
+  float mx[2];
+  if (kQuant) {
+    mx[0] = thread_absmax(rk);
+    mx[1] = thread_absmax(rv);
+    block_max_post(mx, qred);
   }
   // ---- block mean of the keys
   {
@@ -187,6 +195,11 @@ __global__ void __launch_bounds__(256) summary_kv_groups_kernel(const __nv_bfloa
       for (int e = 0; e < 8; ++e) red[warp][0][8 * c16 + e] = ks[e];
     }
     __syncthreads();
+    if (kQuant) {
+      block_max_collect(mx, qred);
+      quant_block_rows(rk, mx[0], f8.k8, f8.sk + (size_t)bh * s.Nb + j, s.N, s.H, b, h, t0, n, tid);
+      if (tid == 0) atomicMax(f8.vmax + bh, __float_as_uint(mx[1]));
+    }
     if (tid < kHeadDim) {
       const int c = tid;
       float sk = 0.f;
