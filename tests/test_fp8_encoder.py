@@ -132,3 +132,16 @@ def test_quantiser_quotient_keeps_exact_midpoints_and_signed_zero(lib):
     q = sa.quot448_host([2.90625, -2.90625, 0.0, -0.0, 3.875], 3.875)
     assert q[0] == 336.0 and q[1] == -336.0 and q[4] == 448.0
     assert q[2] == 0.0 and not np.signbit(q[2]) and q[3] == 0.0 and np.signbit(q[3])
+
+
+def test_quotient_host_entry_validates_its_arguments(lib):
+    import ctypes
+
+    x = (ctypes.c_float * 2)(1.0, 2.0)
+    q = (ctypes.c_float * 2)()
+    assert lib.sol_attn_quot448_host(None, 2, 1.0, q) == -1                 # SOL_ERR_NULL
+    assert lib.sol_attn_quot448_host(x, -1, 1.0, q) == -2                   # SOL_ERR_SHAPE
+    for m in (0.0, -1.0, float("inf"), float("nan")):
+        assert lib.sol_attn_quot448_host(x, 2, m, q) == -10                 # SOL_ERR_OPTION
+    assert lib.sol_attn_quot448_host(x, 0, 1.0, q) == 0
+    assert lib.sol_attn_quot448_host(x, 2, 2.0, q) == 0 and list(q) == [224.0, 448.0]
